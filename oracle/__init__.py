@@ -1,0 +1,10 @@
+"""fp64 CPU oracle for exact attention (test infrastructure only; see attention.py)."""
+
+from .attention import (  # noqa: F401
+    attention_bwd,
+    attention_bwd_head,
+    attention_fwd,
+    attention_fwd_head,
+    attention_fwd_head_tiled,
+    softmax_rows,
+)
