@@ -1,0 +1,233 @@
+"""Fused exact attention for B200 (sm_100a): the Python binding of libfa.so.
+
+The binding marshals arguments only; every step of the computation runs in the CUDA
+kernels behind the C ABI of ``include/fa.h``.  The C entry points are mirrored one to one
+(``fa_fwd``, ``fa_bwd``, ``fa_fwd_ex``, ``fa_bwd_ex``, ``fa_bwd_workspace_bytes``,
+``fa_check_status``, ``fa_status_string``, ``fa_last_launch_count``); they take torch
+tensors (or raw device addresses as ints).  ``attention_forward`` / ``attention_backward``
+and ``FlashAttention`` add output allocation with torch on top.
+
+There is no fallback: if ``libfa.so`` is missing or a call fails, an exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "FAError", "fa_fwd", "fa_bwd", "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_workspace_bytes",
+    "fa_check_status", "fa_status_string", "fa_last_launch_count", "lib", "library_path",
+    "attention_forward", "attention_backward", "FlashAttention", "FA_BF16", "FA_FP16",
+]
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+FA_BF16, FA_FP16 = 0, 1
+TILE = 128
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libfa.so")
+_lib = None
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+
+class FwdArgs(ctypes.Structure):
+    """Mirror of fa_fwd_args."""
+    _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("o", _vp), ("lse", _vp),
+                ("B", _i), ("H", _i), ("N", _i), ("d", _i), ("scale", _f), ("causal", _i),
+                ("blockmask", _vp), ("dtype", _i), ("o_fp32", _i), ("visit_log", _vp),
+                ("stream", _vp)]
+
+
+class BwdArgs(ctypes.Structure):
+    """Mirror of fa_bwd_args."""
+    _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("o", _vp), ("lse", _vp), ("dout", _vp),
+                ("dq", _vp), ("dk", _vp), ("dv", _vp),
+                ("B", _i), ("H", _i), ("N", _i), ("d", _i), ("scale", _f), ("causal", _i),
+                ("blockmask", _vp), ("dtype", _i), ("visit_log", _vp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("stream", _vp)]
+
+
+class FAError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {fa_status_string(code)} ({code})")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfa.so (built in-tree by exact_attention_111_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RuntimeError(f"{library_path} is not built; run `python -m exact_attention_111_b200.build`")
+    L = ctypes.CDLL(library_path)
+    L.fa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp]
+    L.fa_fwd.restype = _i
+    L.fa_bwd.argtypes = [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, ctypes.c_size_t, _vp]
+    L.fa_bwd.restype = _i
+    L.fa_fwd_ex.argtypes = [ctypes.POINTER(FwdArgs)]
+    L.fa_fwd_ex.restype = _i
+    L.fa_bwd_ex.argtypes = [ctypes.POINTER(BwdArgs)]
+    L.fa_bwd_ex.restype = _i
+    L.fa_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
+    L.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+    L.fa_check_status.argtypes = [_vp]
+    L.fa_check_status.restype = _i
+    L.fa_status_string.argtypes = [_i]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_last_launch_count.argtypes = []
+    L.fa_last_launch_count.restype = _i
+    _lib = L
+    return L
+
+
+def _ptr(x):
+    """Device address of a tensor (or None / int passed through)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, what: str):
+    if rc != FA_OK:
+        raise FAError(rc, what)
+
+
+def fa_status_string(code: int) -> str:
+    return lib().fa_status_string(code).decode()
+
+
+def fa_last_launch_count() -> int:
+    return lib().fa_last_launch_count()
+
+
+def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return lib().fa_bwd_workspace_bytes(B, H, N, d)
+
+
+def fa_check_status(stream=None):
+    _check(lib().fa_check_status(_stream(stream)), "fa_check_status")
+
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, blockmask, stream=None):
+    _check(lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
+                        int(bool(causal)), _ptr(blockmask), _stream(stream)), "fa_fwd")
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockmask,
+           workspace, workspace_bytes, stream=None):
+    _check(lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                        _ptr(dk), _ptr(dv), B, H, N, d, scale, int(bool(causal)), _ptr(blockmask),
+                        _ptr(workspace), workspace_bytes, _stream(stream)), "fa_bwd")
+
+
+def fa_fwd_ex(q, k, v, o, lse, B, H, N, d, scale, causal=False, blockmask=None, dtype=FA_BF16,
+              o_fp32=False, visit_log=None, stream=None):
+    a = FwdArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale, int(bool(causal)),
+                _ptr(blockmask), dtype, int(bool(o_fp32)), _ptr(visit_log), _stream(stream))
+    _check(lib().fa_fwd_ex(ctypes.byref(a)), "fa_fwd_ex")
+
+
+def fa_bwd_ex(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal=False, blockmask=None,
+              dtype=FA_BF16, visit_log=None, workspace=None, workspace_bytes=0, stream=None):
+    a = BwdArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                _ptr(dv), B, H, N, d, scale, int(bool(causal)), _ptr(blockmask), dtype,
+                _ptr(visit_log), _ptr(workspace), workspace_bytes, _stream(stream))
+    _check(lib().fa_bwd_ex(ctypes.byref(a)), "fa_bwd_ex")
+
+
+# ----------------------------------------------------------------------------------------
+# torch conveniences (allocation only; the arithmetic is in the kernels)
+# ----------------------------------------------------------------------------------------
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _check_qkv(*ts):
+    for t in ts:
+        if not (t.is_cuda and t.is_contiguous() and t.dim() == 4):
+            raise ValueError("expected contiguous CUDA tensors of shape [B, H, N, d]")
+
+
+def attention_forward(q, k, v, causal=False, blockmask=None, scale=None, o_fp32=False,
+                      visit_log=None, stream=None):
+    """Returns (O, LSE) for [B, H, N, d] CUDA tensors (bf16 or fp16)."""
+    import torch
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    o = torch.empty(q.shape, dtype=torch.float32 if o_fp32 else q.dtype, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fa_fwd_ex(q, k, v, o, lse, B, H, N, d, scale, causal, blockmask, _dtype_code(q), o_fp32,
+              visit_log, stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, dout, causal=False, blockmask=None, scale=None,
+                       workspace=None, visit_log=None, stream=None):
+    """Returns (dQ, dK, dV) for the gradient ``dout`` of O."""
+    import torch
+    _check_qkv(q, k, v, o, dout)
+    B, H, N, d = q.shape
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    nbytes = fa_bwd_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    fa_bwd_ex(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockmask,
+              _dtype_code(q), visit_log, workspace, workspace.numel(), stream)
+    return dq, dk, dv
+
+
+def _make_autograd():
+    import torch
+
+    class FlashAttention(torch.autograd.Function):
+        """autograd glue: forward saves (q, k, v, O, LSE); backward calls fa_bwd."""
+
+        @staticmethod
+        def forward(ctx, q, k, v, causal=False, blockmask=None, scale=None):
+            o, lse = attention_forward(q, k, v, causal, blockmask, scale)
+            ctx.save_for_backward(q, k, v, o, lse)
+            ctx.causal, ctx.blockmask, ctx.scale = causal, blockmask, scale
+            return o
+
+        @staticmethod
+        def backward(ctx, do):
+            q, k, v, o, lse = ctx.saved_tensors
+            dq, dk, dv = attention_backward(q, k, v, o, lse, do.contiguous(), ctx.causal,
+                                            ctx.blockmask, ctx.scale)
+            return dq, dk, dv, None, None, None
+
+    return FlashAttention
+
+
+def __getattr__(name):
+    if name == "FlashAttention":
+        fn = _make_autograd()
+        globals()["FlashAttention"] = fn
+        return fn
+    raise AttributeError(name)

@@ -1,0 +1,486 @@
+// fa_bwd.cu -- fused exact-attention backward pass for sm_100a.
+//
+// The forward saved only O and the per-row log-sum-exp; the backward recomputes every
+// probability tile from Q, K and LSE on chip instead of reading an N x N matrix back
+// (FlashAttention-NeurIPS22 summary, "核心方法 / Backward recomputation").  Gradients of
+// L = sum(dO o O), from the softmax Jacobian:
+//     P = exp(scale*QKᵀ - LSE),  dV = Pᵀ dO,  dP = dO Vᵀ,  D_i = sum_c dO_ic O_ic,
+//     dS = P o (dP - D),  dQ = scale * dS K,  dK = scale * dSᵀ Q.
+//
+// Three kernels on one stream:
+//   bwd_pre   D_i, LSE_i*log2(e) (padded to whole tiles), and a zeroed fp32 dQ accumulator;
+//   bwd_main  one CTA per (b, h, 128-key tile j): K_j, V_j stay in shared memory while the
+//             CTA walks the kept 128-row query tiles i (i >= j under causal masking, and
+//             blockmask[i][j] != 0); dK_j, dV_j accumulate in tensor memory, the dQ_i
+//             partial of each step is added into the fp32 accumulator;
+//   bwd_post  dQ = 16-bit(scale * accumulator).
+//
+// bwd_main roles (320 threads): warps 0-3 one key row per thread (TMEM lanes), warps 4-7
+// drain dQ partials (one query row per thread), warp 8 TMA producer, warp 9 MMA issuer.
+// Tensor memory: Sᵀ/Pᵀ [0,128) (Pᵀ as 16-bit over the first 64 columns), dPᵀ [128,256),
+// dV and dK after them; dQ shares the dPᵀ columns when d = 128 and has its own for d = 64.
+// Per query tile, MMAs in issue order:
+//   Sᵀ = K Q_iᵀ,  dPᵀ = V dO_iᵀ,  dV += Pᵀ dO_i (Pᵀ from TMEM),  dK += dSᵀ Q_i,  dQ_i = dS K
+// where dSᵀ is written once to shared memory (16-bit, 128-byte swizzle) and read both as
+// K-major Sᵀ-shaped operand (for dK) and as its transpose, an MN-major operand (for dQ).
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------------------------
+// bwd_pre
+// ------------------------------------------------------------------------------------
+template <int D, bool kFp16>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreArgs a) {
+  constexpr int G = D / 8;                 // threads per row, 8 elements (16 B) each
+  constexpr int kRowsPerBlock = 256 / G;
+  const int g = threadIdx.x % G;
+  const long long total = (long long)a.BH * a.Np;
+  // Block-uniform trip count: every lane of a warp runs the same iterations (shuffles below).
+  for (long long rb = (long long)blockIdx.x * kRowsPerBlock; rb < total; rb += (long long)gridDim.x * kRowsPerBlock) {
+    const long long r = rb + threadIdx.x / G;
+    const bool active = r < total;
+    const int bh = active ? (int)(r / a.Np) : 0;
+    const int i = active ? (int)(r % a.Np) : a.N;
+    float acc = 0.f;
+    if (i < a.N) {
+      const size_t off = ((size_t)bh * a.N + i) * D + g * 8;
+      const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.o) + off);
+      const uint4 dv = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.dout) + off);
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+      const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 of = unpack2<kFp16>(ow[t]);
+        const float2 df = unpack2<kFp16>(dw[t]);
+        acc = fmaf(of.x, df.x, acc);
+        acc = fmaf(of.y, df.y, acc);
+      }
+      float4* z = reinterpret_cast<float4*>(a.dq_acc + off);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int s = G / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s, G);
+    if (g == 0 && active) {
+      a.delta[r] = acc;
+      float l2 = INFINITY;                     // padding rows and rows with no visible key
+      if (i < a.N) {
+        const float lse = a.lse[(size_t)bh * a.N + i];
+        if (lse > -INFINITY) l2 = lse * kLog2e;
+      }
+      a.lse2[r] = l2;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// bwd_post
+// ------------------------------------------------------------------------------------
+template <bool kFp16>
+__global__ void __launch_bounds__(256) bwd_post_kernel(const BwdPostArgs a) {
+  const long long n8 = a.n_elems / 8;
+  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n8; t += (long long)gridDim.x * blockDim.x) {
+    const float4* src = reinterpret_cast<const float4*>(a.dq_acc) + 2 * t;
+    const float4 x = src[0], y = src[1];
+    uint4 w;
+    w.x = pack2<kFp16>(x.x * a.scale, x.y * a.scale);
+    w.y = pack2<kFp16>(x.z * a.scale, x.w * a.scale);
+    w.z = pack2<kFp16>(y.x * a.scale, y.y * a.scale);
+    w.w = pack2<kFp16>(y.z * a.scale, y.w * a.scale);
+    reinterpret_cast<uint4*>(a.dq)[t] = w;
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// bwd_main
+// ------------------------------------------------------------------------------------
+template <int D>
+struct BwdCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kPanelBytes = kTile * 128;
+  static constexpr int kStages = 2;
+  // layout (offsets from a 1024-byte aligned base)
+  static constexpr int oK = 0;
+  static constexpr int oV = oK + kTileBytes;
+  static constexpr int oQ = oV + kTileBytes;
+  static constexpr int oDO = oQ + kStages * kTileBytes;
+  static constexpr int oDS = oDO + kStages * kTileBytes;     // 128 keys x 128 queries, 16-bit
+  static constexpr int oLSE = oDS + kTile * kTile * 2;
+  static constexpr int oDELTA = oLSE + kStages * kTile * 4;
+  static constexpr int oBAR = oDELTA + kStages * kTile * 4;
+  static constexpr int kSmem = oBAR + 256;
+  static constexpr int tS = 0, tDP = 128, tDV = 256, tDK = 256 + D, tDQ = (D == 128) ? 128 : 384;
+  static constexpr bool kDqSharesDp = (D == 128);
+};
+
+struct BwdBars {
+  uint64_t kv_full;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full, dp_full, p_full, ds_full, dq_full, dq_empty, mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Next query tile at or after i that the key tile j keeps (T when none).
+__device__ __forceinline__ int next_kept(int i, int j, int T, int causal, const uint8_t* mask) {
+  if (causal && i < j) i = j;
+  if (mask != nullptr)
+    while (i < T && __ldg(mask + (size_t)i * T + j) == 0) ++i;
+  return i;
+}
+
+template <int D, bool kFp16>
+__global__ void __launch_bounds__(320, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+               const BwdArgs a) {
+  using C = BwdCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  BwdBars& sh = *reinterpret_cast<BwdBars*>(smem + C::oBAR);
+  const int warp = warp_id(), lane = lane_id();
+  const int bh = blockIdx.x % a.BH;
+  const int j = blockIdx.x / a.BH;                 // key tile; j = 0 first (heaviest under causal)
+  const DevStatus st{a.status, a.timeout_ns};
+  volatile int* abort_flag = &sh.abort_flag;
+  const bool aligned = (smem_addr(smem) & 1023u) == 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sh.kv_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&sh.q_full[s], 1);
+      mbar_init(&sh.q_empty[s], 1);
+    }
+    mbar_init(&sh.s_full, 1);
+    mbar_init(&sh.dp_full, 1);
+    mbar_init(&sh.p_full, 128);
+    mbar_init(&sh.ds_full, 128);
+    mbar_init(&sh.dq_full, 1);
+    mbar_init(&sh.dq_empty, 128);
+    mbar_init(&sh.mma_done, 1);
+    sh.abort_flag = aligned ? 0 : 1;
+    if (!aligned) atomicCAS(a.status, 0, kDevBadState);
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+  const int i_first = next_kept(0, j, a.T, a.causal, a.blockmask);
+  const bool any = aligned && i_first < a.T;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && any) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_do);
+      mbar_arrive_expect_tx(&sh.kv_full, 2 * C::kTileBytes);
+      for (int p = 0; p < C::kPanels; ++p) {
+        tma_load_3d(smem + C::oK + p * C::kPanelBytes, &tm_k, &sh.kv_full, p * 64, j * kTile, bh);
+        tma_load_3d(smem + C::oV + p * C::kPanelBytes, &tm_v, &sh.kv_full, p * 64, j * kTile, bh);
+      }
+      int c = 0;
+      for (int i = i_first; i < a.T; i = next_kept(i + 1, j, a.T, a.causal, a.blockmask), ++c) {
+        const int s = c % C::kStages;
+        if (c >= C::kStages && !mbar_wait(&sh.q_empty[s], ((c / C::kStages) - 1) & 1, abort_flag, st)) break;
+        mbar_arrive_expect_tx(&sh.q_full[s], 2 * C::kTileBytes + 2 * kTile * 4);
+        for (int p = 0; p < C::kPanels; ++p) {
+          tma_load_3d(smem + C::oQ + s * C::kTileBytes + p * C::kPanelBytes, &tm_q, &sh.q_full[s], p * 64, i * kTile, bh);
+          tma_load_3d(smem + C::oDO + s * C::kTileBytes + p * C::kPanelBytes, &tm_do, &sh.q_full[s], p * 64, i * kTile,
+                      bh);
+        }
+        const size_t roff = (size_t)bh * a.Np + (size_t)i * kTile;
+        bulk_load(smem + C::oLSE + s * kTile * 4, a.lse2 + roff, kTile * 4, &sh.q_full[s]);
+        bulk_load(smem + C::oDELTA + s * kTile * 4, a.delta + roff, kTile * 4, &sh.q_full[s]);
+      }
+      if (*abort_flag) {
+        mbar_wait_drain(&sh.kv_full, 0, st);
+        for (int cc = (c > C::kStages ? c - C::kStages : 0); cc < c; ++cc)
+          mbar_wait_drain(&sh.q_full[cc % C::kStages], (cc / C::kStages) & 1, st);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = !any || mbar_wait(&sh.kv_full, 0, abort_flag, st);
+      const uint32_t id_sq = idesc_f16(128, 128, kFp16, false, false);   // K-major x K-major
+      const uint32_t id_kn = idesc_f16(128, D, kFp16, false, true);      // K-major A, MN-major B
+      const uint32_t id_mn = idesc_f16(128, D, kFp16, true, true);       // MN-major A and B
+      const uint32_t aK = smem_addr(smem + C::oK), aV = smem_addr(smem + C::oV);
+      const uint32_t aQ = smem_addr(smem + C::oQ), aDO = smem_addr(smem + C::oDO);
+      const uint32_t aDS = smem_addr(smem + C::oDS);
+      int c = 0;
+      if (any && ok) {
+        for (int i = i_first; i < a.T; i = next_kept(i + 1, j, a.T, a.causal, a.blockmask), ++c) {
+          const int s = c % C::kStages;
+          if (!(ok = mbar_wait(&sh.q_full[s], (c / C::kStages) & 1, abort_flag, st))) break;
+          tc_fence_after();
+          const uint32_t qb = aQ + s * C::kTileBytes, dob = aDO + s * C::kTileBytes;
+          // S^T = K Q_i^T
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+            mma_ss(tmem + C::tS, smem_desc_sw128(aK + koff, 16, 1024), smem_desc_sw128(qb + koff, 16, 1024), id_sq,
+                   kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&sh.s_full);
+          if (a.visit != nullptr) atomicAdd(&a.visit[((size_t)bh * a.T + i) * a.T + j], 1);
+          // dP^T = V dO_i^T  (its columns hold the previous dQ partial when d = 128)
+          if (C::kDqSharesDp && c > 0) {
+            if (!(ok = mbar_wait(&sh.dq_empty, (c - 1) & 1, abort_flag, st))) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+            mma_ss(tmem + C::tDP, smem_desc_sw128(aV + koff, 16, 1024), smem_desc_sw128(dob + koff, 16, 1024), id_sq,
+                   kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&sh.dp_full);
+          // dV += P^T dO_i   (P^T read from tensor memory)
+          if (!(ok = mbar_wait(&sh.p_full, c & 1, abort_flag, st))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + C::tDV, tmem + C::tS + kk * 8, smem_desc_sw128(dob + kk * 2048, C::kPanelBytes, 1024), id_kn,
+                   (c > 0 || kk > 0) ? 1u : 0u);
+          // dK += dS^T Q_i
+          if (!(ok = mbar_wait(&sh.ds_full, c & 1, abort_flag, st))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+            mma_ss(tmem + C::tDK, smem_desc_sw128(aDS + koff, 16, 1024),
+                   smem_desc_sw128(qb + kk * 2048, C::kPanelBytes, 1024), id_kn, (c > 0 || kk > 0) ? 1u : 0u);
+          }
+          // dQ_i = dS K_j   (dS = transpose of the stored dS^T: an MN-major operand)
+          if (!C::kDqSharesDp && c > 0) {
+            if (!(ok = mbar_wait(&sh.dq_empty, (c - 1) & 1, abort_flag, st))) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ss(tmem + C::tDQ, smem_desc_sw128(aDS + kk * 2048, C::kPanelBytes, 1024),
+                   smem_desc_sw128(aK + kk * 2048, C::kPanelBytes, 1024), id_mn, kk > 0 ? 1u : 0u);
+          tc_commit(&sh.dq_full);
+          tc_commit(&sh.q_empty[s]);
+        }
+      }
+      tc_commit(&sh.mma_done);
+      mbar_wait_drain(&sh.mma_done, 0, st);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------------ key-row compute group
+    const int r = warp * 32 + lane;                 // key row within the tile == TMEM lane
+    const int key = j * kTile + r;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + C::tS + lane_off, tDP = tmem + C::tDP + lane_off;
+    const float sl2 = a.scale_log2;
+    const bool key_ok = key < a.N;
+    uint8_t* ds_row = smem + C::oDS + r * 128;
+    int c = 0;
+    bool ok = true;
+    if (any) {
+      for (int i = i_first; i < a.T; i = next_kept(i + 1, j, a.T, a.causal, a.blockmask), ++c) {
+        const int s = c % C::kStages;
+        ok = mbar_wait(&sh.q_full[s], (c / C::kStages) & 1, abort_flag, st) &&
+             mbar_wait(&sh.s_full, c & 1, abort_flag, st);
+        if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+        tc_fence_after();
+        const float* lse2 = reinterpret_cast<const float*>(smem + C::oLSE + s * kTile * 4);
+        const float* dlt = reinterpret_cast<const float*>(smem + C::oDELTA + s * kTile * 4);
+        // keys visible to query q of this tile: key <= q under causal masking
+        const bool diag = a.causal && (i == j);
+        // Phase A: P^T = 2^(scale*log2e*S^T - LSE*log2e), 16-bit, over S^T in TMEM
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t sv[32];
+          tmem_ld32(tS + ch * 32, sv);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const int q0 = ch * 32 + 2 * t;
+            float p0 = ex2(fmaf(__uint_as_float(sv[2 * t]), sl2, -lse2[q0]));
+            float p1 = ex2(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, -lse2[q0 + 1]));
+            if (!key_ok || (diag && r > q0)) p0 = 0.f;
+            if (!key_ok || (diag && r > q0 + 1)) p1 = 0.f;
+            pk[t] = pack2<kFp16>(p0, p1);
+          }
+          tmem_st16(tS + ch * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sh.p_full);
+        // Phase B: dS^T = P^T o (dP^T - D), 16-bit, into shared memory (128-byte swizzle)
+        ok = mbar_wait(&sh.dp_full, c & 1, abort_flag, st) &&
+             (c == 0 || mbar_wait(&sh.dq_full, (c - 1) & 1, abort_flag, st));   // dS^T buffer free
+        if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t dpv[32], pv[16];
+          tmem_ld32(tDP + ch * 32, dpv);
+          tmem_ld16(tS + ch * 16, pv);
+          tmem_wait_ld();
+          uint32_t w[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const int q0 = ch * 32 + 2 * t;
+            const float2 p = unpack2<kFp16>(pv[t]);
+            const float ds0 = p.x * (__uint_as_float(dpv[2 * t]) - dlt[q0]);
+            const float ds1 = p.y * (__uint_as_float(dpv[2 * t + 1]) - dlt[q0 + 1]);
+            w[t] = pack2<kFp16>(ds0, ds1);
+          }
+          // 64 bytes = four 16-byte chunks of this key row, in panel ch/2
+          uint8_t* prow = ds_row + (ch >> 1) * C::kPanelBytes;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int chunk = ((ch & 1) * 4 + t) ^ (r & 7);
+            *reinterpret_cast<uint4*>(prow + chunk * 16) = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sh.ds_full);
+      }
+    }
+    // Epilogue: dV and scale * dK rows of this key tile.
+    if (ok) ok = mbar_wait(&sh.mma_done, 0, abort_flag, st);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const size_t base = ((size_t)bh * a.N + key) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tA = tmem + (which == 0 ? C::tDV : C::tDK) + lane_off;
+        const float f = (which == 0) ? 1.f : a.scale;
+        uint16_t* dst = static_cast<uint16_t*>(which == 0 ? a.dv : a.dk) + base;
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t v[32];
+          if (c > 0) {
+            tmem_ld32(tA + cc, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) v[t] = 0u;
+          }
+          if (key_ok) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              uint4 w;
+              w.x = pack2<kFp16>(__uint_as_float(v[8 * t + 0]) * f, __uint_as_float(v[8 * t + 1]) * f);
+              w.y = pack2<kFp16>(__uint_as_float(v[8 * t + 2]) * f, __uint_as_float(v[8 * t + 3]) * f);
+              w.z = pack2<kFp16>(__uint_as_float(v[8 * t + 4]) * f, __uint_as_float(v[8 * t + 5]) * f);
+              w.w = pack2<kFp16>(__uint_as_float(v[8 * t + 6]) * f, __uint_as_float(v[8 * t + 7]) * f);
+              d4[t] = w;
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ dQ drain group (warps 4-7)
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;                   // query row within the tile == TMEM lane
+    const uint32_t tQ = tmem + C::tDQ + (static_cast<uint32_t>(wq * 32) << 16);
+    int c = 0;
+    if (any) {
+      for (int i = i_first; i < a.T; i = next_kept(i + 1, j, a.T, a.causal, a.blockmask), ++c) {
+        bool ok = mbar_wait(&sh.dq_full, c & 1, abort_flag, st);
+        if (__any_sync(0xffffffffu, !ok)) break;
+        tc_fence_after();
+        const int row = i * kTile + r;
+        float* dst = a.dq_acc + ((size_t)bh * a.N + row) * D;
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t v[32];
+          tmem_ld32(tQ + cc, v);
+          tmem_wait_ld();
+          if (row < a.N) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              atomicAdd(reinterpret_cast<float4*>(dst + cc) + t,
+                        make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
+                                    __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3])));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sh.dq_empty);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool kFp16>
+cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                         const BwdArgs& a, cudaStream_t s) {
+  using C = BwdCfg<D>;
+  auto kern = bwd_kernel<D, kFp16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.T);
+  kern<<<grid, 320, C::kSmem, s>>>(tq, tk, tv, tdo, a);
+  return cudaGetLastError();
+}
+
+int grid_for(long long work_items, int per_block) {
+  long long g = (work_items + per_block - 1) / per_block;
+  const long long cap = 148LL * 16;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return (int)g;
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_pre(const BwdPreArgs& a, bool fp16, cudaStream_t s) {
+  const long long rows = (long long)a.BH * a.Np;
+  if (a.d == 64) {
+    const int g = grid_for(rows, 256 / 8);
+    if (fp16) bwd_pre_kernel<64, true><<<g, 256, 0, s>>>(a);
+    else bwd_pre_kernel<64, false><<<g, 256, 0, s>>>(a);
+  } else {
+    const int g = grid_for(rows, 256 / 16);
+    if (fp16) bwd_pre_kernel<128, true><<<g, 256, 0, s>>>(a);
+    else bwd_pre_kernel<128, false><<<g, 256, 0, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                       const BwdArgs& a, int d, bool fp16, cudaStream_t s) {
+  if (d == 64) return fp16 ? launch_bwd_t<64, true>(tq, tk, tv, tdo, a, s) : launch_bwd_t<64, false>(tq, tk, tv, tdo, a, s);
+  return fp16 ? launch_bwd_t<128, true>(tq, tk, tv, tdo, a, s) : launch_bwd_t<128, false>(tq, tk, tv, tdo, a, s);
+}
+
+cudaError_t launch_bwd_post(const BwdPostArgs& a, bool fp16, cudaStream_t s) {
+  const int g = grid_for(a.n_elems / 8, 256);
+  if (fp16) bwd_post_kernel<true><<<g, 256, 0, s>>>(a);
+  else bwd_post_kernel<false><<<g, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,373 @@
+// fa_fwd.cu -- fused exact-attention forward pass for sm_100a.
+//
+// Computes O = softmax(scale * Q Kᵀ) V and LSE per row in one pass over the key/value
+// tiles, keeping a running row max m and exp-sum l (FlashAttention-NeurIPS22 summary,
+// "核心方法 / Tiling 与 online softmax"); the N x N score and probability tiles live only
+// in tensor memory and registers ("Kernel fusion").  Only O and LSE are written
+// ("Backward recomputation": the forward saves O and the softmax normalisation).
+//
+// One CTA owns two 128-row query tiles of one (b, h) head (256 rows), so every K/V tile
+// it loads feeds two score tiles.  Warp roles (320 threads):
+//   warps 0-3  softmax group 0: query tile 0, one row per thread (TMEM lanes 0..127)
+//   warps 4-7  softmax group 1: query tile 1
+//   warp  8    TMA producer: Q once, then the K/V ring (no multicast)
+//   warp  9    MMA issuer (one elected thread) and TMEM allocator
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 [256+d, 256+2d).
+// P (16-bit) is written over the first 64 columns of its S tile and consumed from TMEM by
+// the PV MMA.  Per key tile u the MMA thread issues, for each query tile q that keeps u:
+//   O_q += P_q(prev) V(prev)   then   S_q = Q_q K(u)ᵀ   (commit -> s_full[q]),
+// so completion of S_q(u) also guarantees O_q holds every earlier PV product: the softmax
+// group may rescale O_q in place before releasing P_q(u).  The row max is refreshed only
+// when it grows by more than 2^8 (exact: the final normalisation uses the same max).
+// The FA-2 idea of spreading one head over SMs ("改进并行性") is the grid over query tiles;
+// its warp repartition to cut shared-memory exchange ("优化块内工作划分") becomes the
+// per-row softmax on TMEM lanes, which needs no cross-warp reduction at all.
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kPanels = D / 64;                 // 64-element (128-byte) swizzle panels
+  static constexpr int kTileBytes = kTile * D * 2;       // one 128 x D 16-bit tile
+  static constexpr int kPanelBytes = kTile * 128;        // 128 rows x 128 bytes
+  static constexpr int kStages = (D == 64) ? 4 : 2;      // K/V ring depth
+  static constexpr int kSmemTiles = 2 * kTileBytes + 2 * kStages * kTileBytes;
+  static constexpr int kThreads = 320;
+};
+
+struct FwdShared {
+  uint64_t q_full;
+  uint64_t k_full[4], v_full[4], kv_empty[4];
+  uint64_t s_full[2], p_full[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+  int n_union;
+  int n_q[2];
+};
+
+constexpr float kLn2 = 0.693147180559945309f;
+constexpr float kRescaleLog2 = 8.0f;   // refresh the running max when it grows by > 2^8
+
+template <int D, bool kFp16>
+__global__ void __launch_bounds__(320, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+  using C = FwdCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ FwdShared sh;
+
+  const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
+  uint8_t* sQ = smem_raw + pad;                           // 2 query tiles
+  uint8_t* sK = sQ + 2 * C::kTileBytes;                   // kStages key tiles
+  uint8_t* sV = sK + C::kStages * C::kTileBytes;          // kStages value tiles
+  int* list = reinterpret_cast<int*>(sV + C::kStages * C::kTileBytes);  // T entries
+
+  const int warp = warp_id(), lane = lane_id();
+  const int bh = blockIdx.x % a.BH;
+  int ui = blockIdx.x / a.BH;
+  if (a.causal) ui = a.n_units - 1 - ui;                  // heaviest query tiles first
+  const int qt0 = 2 * ui;
+  const DevStatus st{a.status, a.timeout_ns};
+  volatile int* abort_flag = &sh.abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sh.q_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&sh.k_full[s], 1);
+      mbar_init(&sh.v_full[s], 1);
+      mbar_init(&sh.kv_empty[s], 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&sh.s_full[q], 1);
+      mbar_init(&sh.p_full[q], 128);
+    }
+    mbar_init(&sh.mma_done, 1);
+    sh.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8) {
+    // Union list of key tiles needed by either query tile, with per-tile keep bits.
+    int count = 0, c0 = 0, c1 = 0;
+    for (int base = 0; base < a.T; base += 32) {
+      const int j = base + lane;
+      bool k0 = false, k1 = false;
+      if (j < a.T) {
+        const int qa = qt0, qb = qt0 + 1;
+        k0 = (!a.causal || j <= qa) && (a.blockmask == nullptr || a.blockmask[(size_t)qa * a.T + j] != 0);
+        k1 = qb < a.T && (!a.causal || j <= qb) &&
+             (a.blockmask == nullptr || a.blockmask[(size_t)qb * a.T + j] != 0);
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, k0 || k1);
+      if (k0 || k1) list[count + __popc(bal & ((1u << lane) - 1u))] = j | (int(k0) << 16) | (int(k1) << 17);
+      count += __popc(bal);
+      c0 += __popc(__ballot_sync(0xffffffffu, k0));
+      c1 += __popc(__ballot_sync(0xffffffffu, k1));
+    }
+    if (lane == 0) {
+      sh.n_union = count;
+      sh.n_q[0] = c0;
+      sh.n_q[1] = c1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+  const int nu = sh.n_union;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && nu > 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      const int nq = (qt0 + 1 < a.T) ? 2 : 1;
+      mbar_arrive_expect_tx(&sh.q_full, nq * C::kTileBytes);
+      for (int q = 0; q < nq; ++q)
+        for (int p = 0; p < C::kPanels; ++p)
+          tma_load_3d(sQ + q * C::kTileBytes + p * C::kPanelBytes, &tm_q, &sh.q_full, p * 64, (qt0 + q) * kTile, bh);
+      int u = 0;
+      for (; u < nu; ++u) {
+        const int s = u % C::kStages;
+        if (u >= C::kStages && !mbar_wait(&sh.kv_empty[s], ((u / C::kStages) - 1) & 1, abort_flag, st)) break;
+        const int j = list[u] & 0xFFFF;
+        mbar_arrive_expect_tx(&sh.k_full[s], C::kTileBytes);
+        for (int p = 0; p < C::kPanels; ++p)
+          tma_load_3d(sK + s * C::kTileBytes + p * C::kPanelBytes, &tm_k, &sh.k_full[s], p * 64, j * kTile, bh);
+        mbar_arrive_expect_tx(&sh.v_full[s], C::kTileBytes);
+        for (int p = 0; p < C::kPanels; ++p)
+          tma_load_3d(sV + s * C::kTileBytes + p * C::kPanelBytes, &tm_v, &sh.v_full[s], p * 64, j * kTile, bh);
+      }
+      if (*abort_flag) {
+        // Let every copy this thread started land before the CTA's shared memory goes away.
+        mbar_wait_drain(&sh.q_full, 0, st);
+        for (int uu = (u > C::kStages ? u - C::kStages : 0); uu < u; ++uu) {
+          mbar_wait_drain(&sh.k_full[uu % C::kStages], (uu / C::kStages) & 1, st);
+          mbar_wait_drain(&sh.v_full[uu % C::kStages], (uu / C::kStages) & 1, st);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = (nu == 0) || mbar_wait(&sh.q_full, 0, abort_flag, st);
+      tc_fence_after();
+      const uint32_t idesc_s = idesc_f16(128, 128, kFp16, false, false);
+      const uint32_t idesc_pv = idesc_f16(128, D, kFp16, false, true);
+      const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
+      int npv[2] = {0, 0};
+      for (int u = 0; u <= nu && ok; ++u) {
+        const int ep = (u > 0) ? list[u - 1] : 0;
+        const int ec = (u < nu) ? list[u] : 0;
+        const int sp = (u + C::kStages - 1) % C::kStages;
+        const int sc = u % C::kStages;
+        bool v_ready = false, k_ready = false;
+        for (int q = 0; q < 2 && ok; ++q) {
+          if (u > 0 && ((ep >> (16 + q)) & 1)) {
+            if (!v_ready) {
+              ok = mbar_wait(&sh.v_full[sp], ((u - 1) / C::kStages) & 1, abort_flag, st);
+              if (!ok) break;
+              v_ready = true;
+            }
+            ok = mbar_wait(&sh.p_full[q], npv[q] & 1, abort_flag, st);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t bdesc = smem_desc_sw128(aV + sp * C::kTileBytes + kk * 2048, C::kPanelBytes, 1024);
+              mma_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8, bdesc, idesc_pv, (npv[q] > 0 || kk > 0) ? 1u : 0u);
+            }
+            ++npv[q];
+          }
+          if (u < nu && ((ec >> (16 + q)) & 1)) {
+            if (!k_ready) {
+              ok = mbar_wait(&sh.k_full[sc], (u / C::kStages) & 1, abort_flag, st);
+              if (!ok) break;
+              tc_fence_after();
+              k_ready = true;
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+              const uint64_t adesc = smem_desc_sw128(aQ + q * C::kTileBytes + koff, 16, 1024);
+              const uint64_t bdesc = smem_desc_sw128(aK + sc * C::kTileBytes + koff, 16, 1024);
+              mma_ss(tmem + q * 128, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&sh.s_full[q]);
+            if (a.visit != nullptr)
+              atomicAdd(&a.visit[((size_t)bh * a.T + (qt0 + q)) * a.T + (ec & 0xFFFF)], 1);
+          }
+        }
+        if (u > 0 && ok) tc_commit(&sh.kv_empty[sp]);
+      }
+      if (ok) {
+        tc_commit(&sh.s_full[0]);   // final phase: every MMA into O_0 / O_1 has completed
+        tc_commit(&sh.s_full[1]);
+      }
+      tc_commit(&sh.mma_done);
+      mbar_wait_drain(&sh.mma_done, 0, st);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax groups
+    const int q = warp >> 2;
+    const int wq = warp & 3;                        // TMEM lane quarter of this warp
+    const int row_local = wq * 32 + lane;
+    const int qt = qt0 + q;
+    const int row = qt * kTile + row_local;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + q * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + q * D + lane_off;
+    const float sl2 = a.scale_log2;
+    float m = -INFINITY;   // running max of scale*log2(e)*s over this row
+    float l = 0.f;         // running sum of 2^(scale*log2(e)*s - m)
+    int c = 0;
+    bool ok = true;
+    for (int u = 0; u < nu; ++u) {
+      const int e = list[u];
+      if (!((e >> (16 + q)) & 1)) continue;
+      const int key0 = (e & 0xFFFF) * kTile;
+      ok = mbar_wait(&sh.s_full[q], c & 1, abort_flag, st);
+      if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_wait_ld();
+      float s[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
+      if ((a.causal && key0 + kTile - 1 > qt * kTile) || key0 + kTile > a.N) {
+        int lim = a.N - key0;                         // keys at or beyond N do not exist
+        if (a.causal) lim = min(lim, row - key0 + 1); // key <= row
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i >= lim) s[i] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      const float mx2 = mx * sl2;
+      float alpha = 1.f;
+      bool resc = false;
+      if (mx2 > m + kRescaleLog2) {
+        alpha = ex2(m - mx2);                       // 0 when m = -inf
+        resc = (c > 0);
+        m = mx2;
+      }
+      const float mneg = (m == -INFINITY) ? 0.f : -m;
+      float sum0 = 0.f, sum1 = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = ex2(fmaf(s[2 * i], sl2, mneg));
+        const float p1 = ex2(fmaf(s[2 * i + 1], sl2, mneg));
+        sum0 += p0;
+        sum1 += p1;
+        pk[i] = pack2<kFp16>(p0, p1);
+      }
+      l = l * alpha + (sum0 + sum1);
+      if (__any_sync(0xffffffffu, resc)) {
+        const float f = resc ? alpha : 1.f;
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+          tmem_st32(tO + cc, o);
+        }
+      }
+      tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sh.p_full[q]);
+      ++c;
+    }
+    // Wait for the final commit: every PV product of this query tile is in O_q.
+    const int nq = sh.n_q[q];
+    if (ok) ok = mbar_wait(&sh.s_full[q], nq & 1, abort_flag, st);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = row < a.N;
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      if (valid) a.lse[(size_t)bh * a.N + row] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+      const size_t obase = ((size_t)bh * a.N + row) * D;
+#pragma unroll
+      for (int cc = 0; cc < D; cc += 32) {
+        uint32_t o[32];
+        if (nq > 0) {
+          tmem_ld32(tO + cc, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        if (valid) {
+          if (a.o_fp32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + obase + cc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                   __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.o) + obase + cc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 w;
+              w.x = pack2<kFp16>(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
+              w.y = pack2<kFp16>(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
+              w.z = pack2<kFp16>(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
+              w.w = pack2<kFp16>(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+              dst[i] = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool kFp16>
+cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdArgs& a,
+                         cudaStream_t s) {
+  using C = FwdCfg<D>;
+  const size_t smem = C::kSmemTiles + (size_t)a.T * sizeof(int) + 1024;
+  auto kern = fwd_kernel<D, kFp16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.n_units);
+  kern<<<grid, C::kThreads, smem, s>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdArgs& a,
+                       int d, bool fp16, cudaStream_t s) {
+  if (d == 64) return fp16 ? launch_fwd_t<64, true>(tq, tk, tv, a, s) : launch_fwd_t<64, false>(tq, tk, tv, a, s);
+  return fp16 ? launch_fwd_t<128, true>(tq, tk, tv, a, s) : launch_fwd_t<128, false>(tq, tk, tv, a, s);
+}
+
+}  // namespace fa

@@ -1,0 +1,257 @@
+// fa_host.cu -- the C ABI of libfa.so (declared in include/fa.h): argument checks, TMA
+// tensor-map encoding, launch sequencing on the caller's stream, status reporting.
+// Every argument check happens before the first CUDA call, so invalid calls fail the
+// same way with or without a GPU.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace fa {
+
+__device__ int g_status_word = 0;
+
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
+thread_local int t_last_launches = 0;
+
+std::mutex g_mu;
+int* g_status_ptr[128] = {nullptr};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bool get_encode() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return true;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return false;
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return true;
+}
+
+// [BH, N, d] 16-bit tensor as a 3-D TMA map with 64 x 128 x 1 boxes, 128-byte swizzle;
+// rows past N read as zero.
+bool encode_qkv(CUtensorMap* m, const void* base, int BH, int N, int d, bool fp16) {
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_shape(int B, int H, int N, int d, float scale, int dtype) {
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
+  if (N > FA_MAX_SEQLEN) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * H > (1LL << 31) - 1) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * H * N * d > (1LL << 46)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct WsLayout {
+  size_t dq_acc, delta, lse2, total;
+};
+
+WsLayout ws_layout(int B, int H, int N, int d) {
+  const size_t BH = (size_t)B * H;
+  const size_t Np = (size_t)((N + kTile - 1) / kTile) * kTile;
+  WsLayout w;
+  w.dq_acc = 0;
+  w.delta = align256(BH * N * d * 4);
+  w.lse2 = w.delta + align256(BH * Np * 4);
+  w.total = w.lse2 + align256(BH * Np * 4);
+  return w;
+}
+
+int status_word(int** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return FA_ERR_CUDA;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_status_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+int* device_status_word() {
+  int* p = nullptr;
+  return status_word(&p) == FA_OK ? p : nullptr;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(int s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+int fa_last_launch_count(void) { return t_last_launches; }
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, 1.f, FA_BF16) != FA_OK) return 0;
+  return ws_layout(B, H, N, d).total;
+}
+
+int fa_fwd_ex(const fa_fwd_args* p) {
+  if (p == nullptr) return FA_ERR_INVALID_ARG;
+  const fa_fwd_args& x = *p;
+  int rc = check_shape(x.B, x.H, x.N, x.d, x.scale, x.dtype);
+  if (rc != FA_OK) return rc;
+  if (!x.q || !x.k || !x.v || !x.o || !x.lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(x.q, 16) || !aligned(x.k, 16) || !aligned(x.v, 16) || !aligned(x.o, 16) || !aligned(x.lse, 4) ||
+      !aligned(x.visit_log, 4))
+    return FA_ERR_INVALID_ARG;
+  const bool fp16 = x.dtype == FA_FP16;
+  const int BH = x.B * x.H;
+  const int T = (x.N + kTile - 1) / kTile;
+  if (!get_encode()) return FA_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (!encode_qkv(&tq, x.q, BH, x.N, x.d, fp16) || !encode_qkv(&tk, x.k, BH, x.N, x.d, fp16) ||
+      !encode_qkv(&tv, x.v, BH, x.N, x.d, fp16))
+    return FA_ERR_CUDA;
+  FwdArgs a{};
+  a.o = x.o;
+  a.lse = x.lse;
+  a.blockmask = x.blockmask;
+  a.visit = x.visit_log;
+  if (status_word(&a.status) != FA_OK) return FA_ERR_CUDA;
+  a.timeout_ns = kWaitLimitNs;
+  a.N = x.N;
+  a.BH = BH;
+  a.T = T;
+  a.n_units = (T + 1) / 2;
+  a.causal = x.causal != 0;
+  a.o_fp32 = x.o_fp32 != 0;
+  a.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
+  t_last_launches = 0;
+  if (launch_fwd(tq, tk, tv, a, x.d, fp16, static_cast<cudaStream_t>(x.stream)) != cudaSuccess) return FA_ERR_CUDA;
+  t_last_launches = 1;
+  return FA_OK;
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d, float scale,
+           int causal, const uint8_t* blockmask, void* stream) {
+  fa_fwd_args a{};
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+  a.B = B; a.H = H; a.N = N; a.d = d;
+  a.scale = scale; a.causal = causal; a.blockmask = blockmask;
+  a.dtype = FA_BF16; a.o_fp32 = 0; a.visit_log = nullptr; a.stream = stream;
+  return fa_fwd_ex(&a);
+}
+
+int fa_bwd_ex(const fa_bwd_args* p) {
+  if (p == nullptr) return FA_ERR_INVALID_ARG;
+  const fa_bwd_args& x = *p;
+  int rc = check_shape(x.B, x.H, x.N, x.d, x.scale, x.dtype);
+  if (rc != FA_OK) return rc;
+  if (!x.q || !x.k || !x.v || !x.o || !x.lse || !x.dout || !x.dq || !x.dk || !x.dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(x.q, 16) || !aligned(x.k, 16) || !aligned(x.v, 16) || !aligned(x.o, 16) || !aligned(x.dout, 16) ||
+      !aligned(x.dq, 16) || !aligned(x.dk, 16) || !aligned(x.dv, 16) || !aligned(x.lse, 4) ||
+      !aligned(x.visit_log, 4))
+    return FA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(x.B, x.H, x.N, x.d);
+  if (!x.workspace || !aligned(x.workspace, 256) || x.workspace_bytes < w.total) return FA_ERR_WORKSPACE;
+  const bool fp16 = x.dtype == FA_FP16;
+  const int BH = x.B * x.H;
+  const int T = (x.N + kTile - 1) / kTile;
+  const int Np = T * kTile;
+  if (!get_encode()) return FA_ERR_CUDA;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_qkv(&tq, x.q, BH, x.N, x.d, fp16) || !encode_qkv(&tk, x.k, BH, x.N, x.d, fp16) ||
+      !encode_qkv(&tv, x.v, BH, x.N, x.d, fp16) || !encode_qkv(&tdo, x.dout, BH, x.N, x.d, fp16))
+    return FA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(x.workspace);
+  float* dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
+  float* delta = reinterpret_cast<float*>(ws + w.delta);
+  float* lse2 = reinterpret_cast<float*>(ws + w.lse2);
+  cudaStream_t s = static_cast<cudaStream_t>(x.stream);
+  int* status = nullptr;
+  if (status_word(&status) != FA_OK) return FA_ERR_CUDA;
+  t_last_launches = 0;
+
+  BwdPreArgs pre{};
+  pre.o = x.o; pre.dout = x.dout; pre.lse = x.lse;
+  pre.delta = delta; pre.lse2 = lse2; pre.dq_acc = dq_acc;
+  pre.N = x.N; pre.Np = Np; pre.BH = BH; pre.d = x.d;
+  if (launch_bwd_pre(pre, fp16, s) != cudaSuccess) return FA_ERR_CUDA;
+
+  BwdArgs b{};
+  b.delta = delta; b.lse2 = lse2; b.dq_acc = dq_acc; b.dk = x.dk; b.dv = x.dv;
+  b.blockmask = x.blockmask; b.visit = x.visit_log; b.status = status; b.timeout_ns = kWaitLimitNs;
+  b.N = x.N; b.Np = Np; b.BH = BH; b.T = T; b.causal = x.causal != 0;
+  b.scale = x.scale;
+  b.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
+  if (launch_bwd(tq, tk, tv, tdo, b, x.d, fp16, s) != cudaSuccess) return FA_ERR_CUDA;
+
+  BwdPostArgs post{};
+  post.dq_acc = dq_acc; post.dq = x.dq; post.n_elems = (long long)BH * x.N * x.d; post.scale = x.scale;
+  if (launch_bwd_post(post, fp16, s) != cudaSuccess) return FA_ERR_CUDA;
+  t_last_launches = 3;
+  return FA_OK;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+           void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, const uint8_t* blockmask,
+           void* workspace, size_t workspace_bytes, void* stream) {
+  fa_bwd_args a{};
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.B = B; a.H = H; a.N = N; a.d = d; a.scale = scale; a.causal = causal; a.blockmask = blockmask;
+  a.dtype = FA_BF16; a.visit_log = nullptr;
+  a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.stream = stream;
+  return fa_bwd_ex(&a);
+}
+
+int fa_check_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int* p = nullptr;
+  if (status_word(&p) != FA_OK) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
+    return v == kDevTimeout ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// fa_internal.h -- argument blocks passed from the host library to the kernels, and the
+// host-side launch functions each kernel file provides.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+constexpr int kTile = 128;          // rows per query tile and keys per key/value tile
+constexpr int kMaxTiles = 2048;     // tile lists live in shared memory (N <= 2048 * 128)
+
+// Error codes a kernel can record in the device status word (read by fa_check_status).
+enum : int { kDevOk = 0, kDevTimeout = 4, kDevBadState = 6 };
+
+struct FwdArgs {
+  void* o;                  // [BH, N, d] 16-bit, or fp32 when o_fp32
+  float* lse;               // [BH, N]
+  const uint8_t* blockmask; // [T, T] or null
+  int* visit;               // [BH, T, T] or null
+  int* status;              // device status word
+  unsigned long long timeout_ns;
+  int N, BH, T, n_units;    // n_units = ceil(T / 2): one CTA covers two 128-row query tiles
+  int causal, o_fp32;
+  float scale_log2;         // scale * log2(e)
+};
+
+struct BwdPreArgs {
+  const void* o;            // [BH, N, d]
+  const void* dout;         // [BH, N, d]
+  const float* lse;         // [BH, N]
+  float* delta;             // [BH, Np]  D_i = sum_c dO_ic O_ic (0 on padding rows)
+  float* lse2;              // [BH, Np]  LSE_i * log2(e) (+inf on padding / empty rows)
+  float* dq_acc;            // [BH, N, d] fp32, zeroed here
+  int N, Np, BH, d;
+};
+
+struct BwdArgs {
+  const float* delta;       // [BH, Np]
+  const float* lse2;        // [BH, Np]
+  float* dq_acc;            // [BH, N, d]
+  void* dk;                 // [BH, N, d] 16-bit
+  void* dv;                 // [BH, N, d] 16-bit
+  const uint8_t* blockmask;
+  int* visit;
+  int* status;
+  unsigned long long timeout_ns;
+  int N, Np, BH, T;
+  int causal;
+  float scale;              // multiplies dK (dQ is scaled in the post pass)
+  float scale_log2;
+};
+
+struct BwdPostArgs {
+  const float* dq_acc;      // [BH, N, d]
+  void* dq;                 // [BH, N, d] 16-bit
+  long long n_elems;
+  float scale;
+};
+
+// Launchers (defined next to each kernel).  Return a cudaError_t.
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdArgs& a,
+                       int d, bool fp16, cudaStream_t s);
+cudaError_t launch_bwd_pre(const BwdPreArgs& a, bool fp16, cudaStream_t s);
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const BwdArgs& a, int d, bool fp16, cudaStream_t s);
+cudaError_t launch_bwd_post(const BwdPostArgs& a, bool fp16, cudaStream_t s);
+
+int* device_status_word();  // address of the per-process device status word
+
+}  // namespace fa
