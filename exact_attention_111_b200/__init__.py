@@ -48,7 +48,8 @@ class BwdArgs(ctypes.Structure):
                 ("dq", _vp), ("dk", _vp), ("dv", _vp),
                 ("B", _i), ("H", _i), ("N", _i), ("d", _i), ("scale", _f), ("causal", _i),
                 ("blockmask", _vp), ("dtype", _i), ("visit_log", _vp),
-                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("stream", _vp)]
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("stream", _vp),
+                ("main_start_event", _vp), ("main_stop_event", _vp)]
 
 
 class FAError(RuntimeError):
@@ -143,11 +144,19 @@ def fa_fwd_ex(q, k, v, o, lse, B, H, N, d, scale, causal=False, blockmask=None, 
     _check(lib().fa_fwd_ex(ctypes.byref(a)), "fa_fwd_ex")
 
 
+def _event(e):
+    if e is None or isinstance(e, int):
+        return e
+    return e.cuda_event  # torch.cuda.Event (created lazily by torch on first use)
+
+
 def fa_bwd_ex(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal=False, blockmask=None,
-              dtype=FA_BF16, visit_log=None, workspace=None, workspace_bytes=0, stream=None):
+              dtype=FA_BF16, visit_log=None, workspace=None, workspace_bytes=0, stream=None,
+              main_start_event=None, main_stop_event=None):
     a = BwdArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
                 _ptr(dv), B, H, N, d, scale, int(bool(causal)), _ptr(blockmask), dtype,
-                _ptr(visit_log), _ptr(workspace), workspace_bytes, _stream(stream))
+                _ptr(visit_log), _ptr(workspace), workspace_bytes, _stream(stream),
+                _event(main_start_event), _event(main_stop_event))
     _check(lib().fa_bwd_ex(ctypes.byref(a)), "fa_bwd_ex")
 
 

@@ -219,7 +219,11 @@ int fa_bwd_ex(const fa_bwd_args* p) {
   b.N = x.N; b.Np = Np; b.BH = BH; b.T = T; b.causal = x.causal != 0;
   b.scale = x.scale;
   b.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
+  if (x.main_start_event && cudaEventRecord(static_cast<cudaEvent_t>(x.main_start_event), s) != cudaSuccess)
+    return FA_ERR_CUDA;
   if (launch_bwd(tq, tk, tv, tdo, b, x.d, fp16, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (x.main_stop_event && cudaEventRecord(static_cast<cudaEvent_t>(x.main_stop_event), s) != cudaSuccess)
+    return FA_ERR_CUDA;
 
   BwdPostArgs post{};
   post.dq_acc = dq_acc; post.dq = x.dq; post.n_elems = (long long)BH * x.N * x.d; post.scale = x.scale;

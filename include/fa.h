@@ -110,6 +110,9 @@ typedef struct {
   int* visit_log;          /* as in fa_fwd_args, for the main backward kernel        */
   void* workspace; size_t workspace_bytes;
   void* stream;
+  void* main_start_event;  /* NULL, or a cudaEvent_t recorded on `stream` right before the
+                              fused main backward kernel (for per-kernel timing)       */
+  void* main_stop_event;   /* NULL, or a cudaEvent_t recorded right after it           */
 } fa_bwd_args;
 
 int fa_fwd_ex(const fa_fwd_args* args);

@@ -99,6 +99,18 @@ def test_forward_workloads_sampled(name):
         assert np.array_equal(vl.cpu().numpy(), P.expected_visits(w.B, w.H, w.N, False, mask.numpy()))
 
 
+def test_forward_long_context_fp32_output_strict():
+    """The peaked long-context workload (K scaled by 4, causal, N = 16384, d = 128) with fp32
+    O: max |O - O_ref| <= 1e-2 with no output-rounding allowance, on sampled whole heads."""
+    w = workloads()["long_B1_H32_N16384_d128_causal_k4"]
+    inp = P.inputs(w.B, w.H, w.N, w.d, w.seed, k_scale=w.k_scale)
+    o, lse, _ = P.gpu_forward(inp, True, None, o_fp32=True)
+    heads = P.sample_heads(w.B, w.H, 4, seed=w.seed + 1)
+    o_ref, lse_ref = P.oracle_forward(inp, True, None, heads=heads)
+    worst_o, worst_l = P.check_forward(o, lse, o_ref, lse_ref, heads=heads, o16_dtype=None, label="long fp32 O")
+    print(f"long-context fp32 O: max |O err| {worst_o:.4g}, max |LSE err| {worst_l:.4g}")
+
+
 def test_forward_deterministic():
     inp = P.inputs(2, 4, 2000, 128, seed=15)
     o1, l1, _ = P.gpu_forward(inp, True, None)
