@@ -17,8 +17,10 @@
 // the PV MMA.  Per key tile u the MMA thread issues, for each query tile q that keeps u:
 //   O_q += P_q(prev) V(prev)   then   S_q = Q_q K(u)ᵀ   (commit -> s_full[q]),
 // so completion of S_q(u) also guarantees O_q holds every earlier PV product: the softmax
-// group may rescale O_q in place before releasing P_q(u).  The row max is refreshed only
-// when it grows by more than 2^8 (exact: the final normalisation uses the same max).
+// group may rescale O_q in place before releasing P_q(u).  The row max is refreshed whenever
+// it grows, so the largest probability of a row is exactly 1 when it is rounded to 16 bits
+// (a stale max would leave it anywhere in [1, 2^k) and add up to 2^-8 relative rounding on the
+// dominant term of peaked rows).
 // The FA-2 idea of spreading one head over SMs ("改进并行性") is the grid over query tiles;
 // its warp repartition to cut shared-memory exchange ("优化块内工作划分") becomes the
 // per-row softmax on TMEM lanes, which needs no cross-warp reduction at all.
@@ -50,7 +52,6 @@ struct FwdShared {
 };
 
 constexpr float kLn2 = 0.693147180559945309f;
-constexpr float kRescaleLog2 = 8.0f;   // refresh the running max when it grows by > 2^8
 
 template <int D, bool kFp16>
 __global__ void __launch_bounds__(320, 1)
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(320, 1)
       const float mx2 = mx * sl2;
       float alpha = 1.f;
       bool resc = false;
-      if (mx2 > m + kRescaleLog2) {
+      if (mx2 > m) {
         alpha = ex2(m - mx2);                       // 0 when m = -inf
         resc = (c > 0);
         m = mx2;
