@@ -17,7 +17,7 @@ import os
 
 __all__ = [
     "FAError", "fa_fwd", "fa_bwd", "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_workspace_bytes",
-    "fa_check_status", "fa_status_string", "fa_last_launch_count", "lib", "library_path",
+    "fa_check_status", "fa_status_string", "fa_last_launch_count", "fa_bwd_noalloc", "lib", "library_path",
     "attention_forward", "attention_backward", "FlashAttention", "FA_BF16", "FA_FP16",
 ]
 
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.fa_check_status.restype = _i
     L.fa_status_string.argtypes = [_i]
     L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_bwd_noalloc.argtypes = [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp]
+    L.fa_bwd_noalloc.restype = _i
     L.fa_last_launch_count.argtypes = []
     L.fa_last_launch_count.restype = _i
     _lib = L
@@ -135,6 +137,15 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockma
     _check(lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
                         _ptr(dk), _ptr(dv), B, H, N, d, scale, int(bool(causal)), _ptr(blockmask),
                         _ptr(workspace), workspace_bytes, _stream(stream)), "fa_bwd")
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockmask,
+                   stream=None):
+    """fa_bwd without a workspace argument, for callers that cannot allocate device memory
+    at call time; uses the library's fixed 64 MiB per-device scratch (see include/fa.h)."""
+    _check(lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                                _ptr(dk), _ptr(dv), B, H, N, d, scale, int(bool(causal)),
+                                _ptr(blockmask), _stream(stream)), "fa_bwd_noalloc")
 
 
 def fa_fwd_ex(q, k, v, o, lse, B, H, N, d, scale, causal=False, blockmask=None, dtype=FA_BF16,

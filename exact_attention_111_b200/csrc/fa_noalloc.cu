@@ -1,0 +1,64 @@
+// fa_noalloc.cu -- fa_bwd_noalloc: the backward pass for callers that cannot allocate
+// device memory at call time.
+//
+// fa_bwd needs a caller-provided scratch buffer (fp32 dQ accumulator and two per-row
+// vectors).  Some callers have no way to provide one when they call: an inference- or
+// training-engine plugin whose enqueue step must not allocate, a host program that links
+// libfa.so without any device allocator of its own, or code running while the process's
+// device memory pool is frozen.  For them this file holds the scratch in a fixed
+// file-scope device array instead, and the entry point allocates nothing.
+//
+// The array (kNoAllocScratchBytes) exists on every GPU that loads the library, until the
+// process exits.  Every call on a device shares that device's array, so calls that overlap
+// on the GPU (other streams, other host threads) race on it and must be serialised by the
+// caller.  The array keeps the last call's contents; the backward's first kernel rewrites
+// every part the later kernels read (it zeroes the dQ accumulator and writes both per-row
+// vectors), so nothing has to be cleared between calls.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)FA_NOALLOC_SCRATCH_BYTES;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[128] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device.  In host code the array's name
+// is only a host-side stand-in, so the address is asked from the runtime once per device.
+int scratch_for_current_device(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                              const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                              float scale, int causal, const uint8_t* blockmask, void* stream) {
+  const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
+  if (need == 0) {
+    // invalid shape: let the regular entry point report the precise argument error
+    return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockmask, nullptr, 0, stream);
+  }
+  if (need > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const int rc = scratch_for_current_device(&scratch);
+  if (rc != FA_OK) return rc;
+  return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockmask, scratch,
+                kNoAllocScratchBytes, stream);
+}

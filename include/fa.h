@@ -124,6 +124,37 @@ int fa_bwd_ex(const fa_bwd_args* args);
  */
 int fa_check_status(void* stream);
 
+/* Size of the fixed device scratch array that fa_bwd_noalloc uses: 64 MiB. */
+#define FA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * fa_bwd_noalloc -- fa_bwd for callers that cannot allocate device memory when they call.
+ * (No counterpart in the paper: this is a deployment variant of the backward entry point.)
+ *
+ * Who needs it: callers with no device allocator at call time, such as an engine plugin
+ * whose enqueue step must not allocate, a host program linking libfa.so without any device
+ * allocator of its own, or code running while the device memory pool is frozen.  fa_bwd
+ * asks them for a workspace they cannot provide; this entry point instead uses one fixed
+ * file-scope device array of FA_NOALLOC_SCRATCH_BYTES that lives on every GPU that loads
+ * the library until the process exits.
+ *
+ * Arguments and results are exactly those of fa_bwd without the workspace pair.
+ * Limits and behaviour:
+ *   - returns FA_ERR_WORKSPACE, launching nothing, when fa_bwd_workspace_bytes(B, H, N, d)
+ *     exceeds FA_NOALLOC_SCRATCH_BYTES (roughly B*H*N*(4*d + 8) bytes must fit in 64 MiB);
+ *   - allocates nothing: no cudaMalloc / cudaFree and no allocating library routine;
+ *   - the first call on a device looks up the array's device address for that device
+ *     (cudaGetSymbolAddress); make that first call before any stream capture;
+ *   - every call on a device shares the one array, which keeps the last call's contents
+ *     (the backward rewrites all of it that it reads, so nothing needs clearing); calls that
+ *     overlap on the GPU -- other streams or host threads -- race on it, so the caller
+ *     must serialise them.
+ */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dout, void* dq, void* dk, void* dv,
+                   int B, int H, int N, int d, float scale, int causal, const uint8_t* blockmask,
+                   void* stream);
+
 /* Static human-readable name of a status code. */
 const char* fa_status_string(int status);
 
