@@ -144,13 +144,25 @@ def dist_setup():
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank device time over all ranks (NCCL on GPUs, gloo in CPU tests)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch of heads (weak scaling over independent heads)."""
+    return base_seed + 7919 * rank
+
+
+def aggregate_tflops(world: int, flops_per_rank_step: float, steps: int, max_elapsed_ms: float) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's device time."""
+    return world * flops_per_rank_step * steps / (max_elapsed_ms * 1e-3) / 1e12
 
 
 def barrier(world: int):
@@ -237,7 +249,7 @@ def run_ours(args, w, world, rank, local):
     fa.lib()  # fails loudly when the CUDA library is missing
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
-    inp = make_inputs(w.B, w.H, w.N, w.d, w.seed + 7919 * rank, k_scale=w.k_scale)
+    inp = make_inputs(w.B, w.H, w.N, w.d, rank_seed(w.seed, rank), k_scale=w.k_scale)
     host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "dout")}
     d = {n: t.to(dev) for n, t in host.items()}
     mask = butterfly_blockmask(w.tiles).to(dev) if w.butterfly else None
@@ -307,7 +319,7 @@ def run_ours(args, w, world, rank, local):
     step_flops = attention_flops(B, H, N, D, w.causal, True)
     bwd_flops = step_flops - fwd_flops
     ms_step = elapsed_ms / args.steps
-    value = world * step_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = aggregate_tflops(world, step_flops, args.steps, elapsed_ms)
     fwd_ms = statistics.mean(per_kernel["fwd"])
     bmain_ms = statistics.mean(per_kernel["bwd_main"])
     fwd_tflops = fwd_flops / (fwd_ms * 1e-3) / 1e12
@@ -340,7 +352,7 @@ def run_ours(args, w, world, rank, local):
     t2.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(s2.elapsed_time(t2), world)
-    e2e_value = world * step_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_value = aggregate_tflops(world, step_flops, e2e_steps, e2e_ms)
     fa.fa_check_status(stream)
 
     if rank != 0:
