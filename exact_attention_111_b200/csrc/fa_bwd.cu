@@ -15,12 +15,13 @@
 //             partial of each step is added into the fp32 accumulator;
 //   bwd_post  dQ = 16-bit(scale * accumulator).
 //
-// bwd_main roles (320 threads): warps 0-3 one key row per thread (TMEM lanes), warps 4-7
-// drain dQ partials (one query row per thread), warp 8 TMA producer, warp 9 MMA issuer.
+// bwd_main roles (448 threads): warps 0-7 two compute groups, one key row per thread (TMEM
+// lanes), each group owning half of the query columns; warps 8-11 drain dQ partials (one
+// query row per thread); warp 12 TMA producer; warp 13 MMA issuer.
 // Tensor memory: Sᵀ/Pᵀ [0,128) (Pᵀ as 16-bit over the first 64 columns), dPᵀ [128,256),
 // dV and dK after them; dQ shares the dPᵀ columns when d = 128 and has its own for d = 64.
-// Per query tile, MMAs in issue order:
-//   Sᵀ = K Q_iᵀ,  dPᵀ = V dO_iᵀ,  dV += Pᵀ dO_i (Pᵀ from TMEM),  dK += dSᵀ Q_i,  dQ_i = dS K
+// Per query tile, the MMAs: Sᵀ = K Q_iᵀ, dPᵀ = V dO_iᵀ, dV += Pᵀ dO_i (Pᵀ from TMEM),
+// dK += dSᵀ Q_i, dQ_i = dS K, issued one tile ahead where TMEM allows (see the MMA role)
 // where dSᵀ is written once to shared memory (16-bit, 128-byte swizzle) and read both as
 // K-major Sᵀ-shaped operand (for dK) and as its transpose, an MN-major operand (for dQ).
 #include "fa_internal.h"
@@ -119,6 +120,10 @@ struct BwdCfg {
   static constexpr bool kDqSharesDp = (D == 128);
 };
 
+constexpr int kBwdThreads = 448;   // 2 compute groups, dQ drain group, producer, MMA
+constexpr int kBwdLoadWarp = 12;
+constexpr int kBwdMmaWarp = 13;
+
 struct BwdBars {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2];
@@ -136,7 +141,7 @@ __device__ __forceinline__ int next_kept(int i, int j, int T, int causal, const 
 }
 
 template <int D, bool kFp16>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const BwdArgs a) {
@@ -158,8 +163,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(&sh.s_full, 1);
     mbar_init(&sh.dp_full, 1);
-    mbar_init(&sh.p_full, 128);
-    mbar_init(&sh.ds_full, 128);
+    mbar_init(&sh.p_full, 256);
+    mbar_init(&sh.ds_full, 256);
     mbar_init(&sh.dq_full, 1);
     mbar_init(&sh.dq_empty, 128);
     mbar_init(&sh.mma_done, 1);
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(320, 1)
     if (!aligned) atomicCAS(a.status, 0, kDevBadState);
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == kBwdMmaWarp) {
     tmem_alloc(&sh.tmem_base, 512);
     tmem_relinquish();
   }
@@ -178,7 +183,7 @@ __global__ void __launch_bounds__(320, 1)
   const int i_first = next_kept(0, j, a.T, a.causal, a.blockmask);
   const bool any = aligned && i_first < a.T;
 
-  if (warp == 8) {
+  if (warp == kBwdLoadWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && any) {
       prefetch_tmap(&tm_q);
@@ -211,52 +216,69 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == kBwdMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
+    // Issue order per kept query tile c (stage s = c % 2):
+    //   [Sᵀ(c), dPᵀ(c) issued one step earlier]  dV += Pᵀ(c) dO(c);  Sᵀ(c+1);
+    //   dK += dSᵀ(c) Q(c);  dQ(c) = dS(c) K;  dPᵀ(c+1)
+    // so Sᵀ(c+1) runs while the compute groups form dS(c), and dPᵀ(c+1) while they form P(c+1).
+    // Sᵀ(c+1) overwrites Pᵀ(c) in TMEM only after dV(c), which reads it, was issued
+    // (tcgen05.mma operations from one thread execute in issue order).
     if (lane == 0) {
-      bool ok = !any || mbar_wait(&sh.kv_full, 0, abort_flag, st);
       const uint32_t id_sq = idesc_f16(128, 128, kFp16, false, false);   // K-major x K-major
       const uint32_t id_kn = idesc_f16(128, D, kFp16, false, true);      // K-major A, MN-major B
       const uint32_t id_mn = idesc_f16(128, D, kFp16, true, true);       // MN-major A and B
       const uint32_t aK = smem_addr(smem + C::oK), aV = smem_addr(smem + C::oV);
       const uint32_t aQ = smem_addr(smem + C::oQ), aDO = smem_addr(smem + C::oDO);
       const uint32_t aDS = smem_addr(smem + C::oDS);
+      auto issue_s = [&](int s) {   // Sᵀ = K Q_sᵀ
+        const uint32_t qb = aQ + s * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+          mma_ss(tmem + C::tS, smem_desc_sw128(aK + koff, 16, 1024), smem_desc_sw128(qb + koff, 16, 1024), id_sq,
+                 kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&sh.s_full);
+      };
+      auto issue_dp = [&](int s) {  // dPᵀ = V dO_sᵀ
+        const uint32_t dob = aDO + s * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+          mma_ss(tmem + C::tDP, smem_desc_sw128(aV + koff, 16, 1024), smem_desc_sw128(dob + koff, 16, 1024), id_sq,
+                 kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&sh.dp_full);
+      };
+      bool ok = any && mbar_wait(&sh.kv_full, 0, abort_flag, st) && mbar_wait(&sh.q_full[0], 0, abort_flag, st);
       int c = 0;
-      if (any && ok) {
-        for (int i = i_first; i < a.T; i = next_kept(i + 1, j, a.T, a.causal, a.blockmask), ++c) {
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        if (a.visit != nullptr) atomicAdd(&a.visit[((size_t)bh * a.T + i_first) * a.T + j], 1);
+        issue_dp(0);
+        for (int i = i_first; i < a.T; ++c) {
           const int s = c % C::kStages;
-          if (!(ok = mbar_wait(&sh.q_full[s], (c / C::kStages) & 1, abort_flag, st))) break;
-          tc_fence_after();
+          const int i_next = next_kept(i + 1, j, a.T, a.causal, a.blockmask);
+          const bool more = i_next < a.T;
           const uint32_t qb = aQ + s * C::kTileBytes, dob = aDO + s * C::kTileBytes;
-          // S^T = K Q_i^T
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-            mma_ss(tmem + C::tS, smem_desc_sw128(aK + koff, 16, 1024), smem_desc_sw128(qb + koff, 16, 1024), id_sq,
-                   kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&sh.s_full);
-          if (a.visit != nullptr) atomicAdd(&a.visit[((size_t)bh * a.T + i) * a.T + j], 1);
-          // dP^T = V dO_i^T  (its columns hold the previous dQ partial when d = 128)
-          if (C::kDqSharesDp && c > 0) {
-            if (!(ok = mbar_wait(&sh.dq_empty, (c - 1) & 1, abort_flag, st))) break;
-            tc_fence_after();
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-            mma_ss(tmem + C::tDP, smem_desc_sw128(aV + koff, 16, 1024), smem_desc_sw128(dob + koff, 16, 1024), id_sq,
-                   kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&sh.dp_full);
-          // dV += P^T dO_i   (P^T read from tensor memory)
+          // dV += Pᵀ dO(c)   (Pᵀ read from tensor memory)
           if (!(ok = mbar_wait(&sh.p_full, c & 1, abort_flag, st))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
             mma_ts(tmem + C::tDV, tmem + C::tS + kk * 8, smem_desc_sw128(dob + kk * 2048, C::kPanelBytes, 1024), id_kn,
                    (c > 0 || kk > 0) ? 1u : 0u);
-          // dK += dS^T Q_i
+          // Sᵀ(c+1)
+          if (more) {
+            const int s1 = (c + 1) % C::kStages;
+            if (!(ok = mbar_wait(&sh.q_full[s1], ((c + 1) / C::kStages) & 1, abort_flag, st))) break;
+            tc_fence_after();
+            issue_s(s1);
+            if (a.visit != nullptr) atomicAdd(&a.visit[((size_t)bh * a.T + i_next) * a.T + j], 1);
+          }
+          // dK += dSᵀ Q(c)
           if (!(ok = mbar_wait(&sh.ds_full, c & 1, abort_flag, st))) break;
           tc_fence_after();
 #pragma unroll
@@ -265,7 +287,7 @@ __global__ void __launch_bounds__(320, 1)
             mma_ss(tmem + C::tDK, smem_desc_sw128(aDS + koff, 16, 1024),
                    smem_desc_sw128(qb + kk * 2048, C::kPanelBytes, 1024), id_kn, (c > 0 || kk > 0) ? 1u : 0u);
           }
-          // dQ_i = dS K_j   (dS = transpose of the stored dS^T: an MN-major operand)
+          // dQ(c) = dS K   (dS = transpose of the stored dSᵀ: an MN-major operand)
           if (!C::kDqSharesDp && c > 0) {
             if (!(ok = mbar_wait(&sh.dq_empty, (c - 1) & 1, abort_flag, st))) break;
             tc_fence_after();
@@ -276,21 +298,34 @@ __global__ void __launch_bounds__(320, 1)
                    smem_desc_sw128(aK + kk * 2048, C::kPanelBytes, 1024), id_mn, kk > 0 ? 1u : 0u);
           tc_commit(&sh.dq_full);
           tc_commit(&sh.q_empty[s]);
+          // dPᵀ(c+1)   (its columns hold dQ(c) when d = 128: wait for the drain)
+          if (more) {
+            if (C::kDqSharesDp) {
+              if (!(ok = mbar_wait(&sh.dq_empty, c & 1, abort_flag, st))) break;
+              tc_fence_after();
+            }
+            issue_dp((c + 1) % C::kStages);
+          }
+          i = i_next;
         }
       }
       tc_commit(&sh.mma_done);
       mbar_wait_drain(&sh.mma_done, 0, st);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------------------------------------ key-row compute group
-    const int r = warp * 32 + lane;                 // key row within the tile == TMEM lane
+  } else if (warp < 8) {
+    // ------------------------------------------------------------------ key-row compute groups
+    // Group g (warps 4g..4g+3) owns query columns [64g, 64g+64) of every Sᵀ / dPᵀ tile; each
+    // thread owns one key row (TMEM lane).  P stays in registers between the two phases.
+    const int g = warp >> 2;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;                   // key row within the tile == TMEM lane
     const int key = j * kTile + r;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + C::tS + lane_off, tDP = tmem + C::tDP + lane_off;
     const float sl2 = a.scale_log2;
     const bool key_ok = key < a.N;
-    uint8_t* ds_row = smem + C::oDS + r * 128;
+    uint8_t* ds_row = smem + C::oDS + g * C::kPanelBytes + r * 128;
     int c = 0;
     bool ok = true;
     if (any) {
@@ -300,57 +335,55 @@ __global__ void __launch_bounds__(320, 1)
              mbar_wait(&sh.s_full, c & 1, abort_flag, st);
         if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
         tc_fence_after();
-        const float* lse2 = reinterpret_cast<const float*>(smem + C::oLSE + s * kTile * 4);
-        const float* dlt = reinterpret_cast<const float*>(smem + C::oDELTA + s * kTile * 4);
-        // keys visible to query q of this tile: key <= q under causal masking
-        const bool diag = a.causal && (i == j);
-        // Phase A: P^T = 2^(scale*log2e*S^T - LSE*log2e), 16-bit, over S^T in TMEM
+        const float* lse2 = reinterpret_cast<const float*>(smem + C::oLSE + s * kTile * 4) + 64 * g;
+        const float* dlt = reinterpret_cast<const float*>(smem + C::oDELTA + s * kTile * 4) + 64 * g;
+        const bool diag = a.causal && (i == j);     // key r visible to query column q iff r <= q
+        // Phase A: Pᵀ = 2^(scale*log2e*Sᵀ - LSE*log2e), 16-bit, over Sᵀ in TMEM
+        uint32_t pk[32];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int h = 0; h < 2; ++h) {
           uint32_t sv[32];
-          tmem_ld32(tS + ch * 32, sv);
+          tmem_ld32(tS + 64 * g + 32 * h, sv);
           tmem_wait_ld();
-          uint32_t pk[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
-            const int q0 = ch * 32 + 2 * t;
-            float p0 = ex2(fmaf(__uint_as_float(sv[2 * t]), sl2, -lse2[q0]));
-            float p1 = ex2(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, -lse2[q0 + 1]));
+            const int ql = 32 * h + 2 * t;          // column within this group's 64
+            const int q0 = 64 * g + ql;             // column within the tile
+            float p0 = ex2(fmaf(__uint_as_float(sv[2 * t]), sl2, -lse2[ql]));
+            float p1 = ex2(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, -lse2[ql + 1]));
             if (!key_ok || (diag && r > q0)) p0 = 0.f;
             if (!key_ok || (diag && r > q0 + 1)) p1 = 0.f;
-            pk[t] = pack2<kFp16>(p0, p1);
+            pk[16 * h + t] = pack2<kFp16>(p0, p1);
           }
-          tmem_st16(tS + ch * 16, pk);
         }
+        tmem_st32(tS + 32 * g, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sh.p_full);
-        // Phase B: dS^T = P^T o (dP^T - D), 16-bit, into shared memory (128-byte swizzle)
+        // Phase B: dSᵀ = Pᵀ o (dPᵀ - D), 16-bit, into this group's shared-memory panel
         ok = mbar_wait(&sh.dp_full, c & 1, abort_flag, st) &&
-             (c == 0 || mbar_wait(&sh.dq_full, (c - 1) & 1, abort_flag, st));   // dS^T buffer free
+             (c == 0 || mbar_wait(&sh.dq_full, (c - 1) & 1, abort_flag, st));   // dSᵀ buffer free
         if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t dpv[32], pv[16];
-          tmem_ld32(tDP + ch * 32, dpv);
-          tmem_ld16(tS + ch * 16, pv);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t dpv[32];
+          tmem_ld32(tDP + 64 * g + 32 * h, dpv);
           tmem_wait_ld();
           uint32_t w[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
-            const int q0 = ch * 32 + 2 * t;
-            const float2 p = unpack2<kFp16>(pv[t]);
-            const float ds0 = p.x * (__uint_as_float(dpv[2 * t]) - dlt[q0]);
-            const float ds1 = p.y * (__uint_as_float(dpv[2 * t + 1]) - dlt[q0 + 1]);
+            const int ql = 32 * h + 2 * t;
+            const float2 p = unpack2<kFp16>(pk[16 * h + t]);
+            const float ds0 = p.x * (__uint_as_float(dpv[2 * t]) - dlt[ql]);
+            const float ds1 = p.y * (__uint_as_float(dpv[2 * t + 1]) - dlt[ql + 1]);
             w[t] = pack2<kFp16>(ds0, ds1);
           }
-          // 64 bytes = four 16-byte chunks of this key row, in panel ch/2
-          uint8_t* prow = ds_row + (ch >> 1) * C::kPanelBytes;
+          // 64 bytes = four 16-byte chunks of this key row (128-byte swizzle)
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
-            const int chunk = ((ch & 1) * 4 + t) ^ (r & 7);
-            *reinterpret_cast<uint4*>(prow + chunk * 16) = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
+            const int chunk = (h * 4 + t) ^ (r & 7);
+            *reinterpret_cast<uint4*>(ds_row + chunk * 16) = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
           }
         }
         fence_async_smem();
@@ -358,44 +391,41 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(&sh.ds_full);
       }
     }
-    // Epilogue: dV and scale * dK rows of this key tile.
+    // Epilogue: group 0 writes dV, group 1 writes scale * dK, one key row per thread.
     if (ok) ok = mbar_wait(&sh.mma_done, 0, abort_flag, st);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
       const size_t base = ((size_t)bh * a.N + key) * D;
+      const uint32_t tA = tmem + (g == 0 ? C::tDV : C::tDK) + lane_off;
+      const float f = (g == 0) ? 1.f : a.scale;
+      uint16_t* dst = static_cast<uint16_t*>(g == 0 ? a.dv : a.dk) + base;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t tA = tmem + (which == 0 ? C::tDV : C::tDK) + lane_off;
-        const float f = (which == 0) ? 1.f : a.scale;
-        uint16_t* dst = static_cast<uint16_t*>(which == 0 ? a.dv : a.dk) + base;
+      for (int cc = 0; cc < D; cc += 32) {
+        uint32_t v[32];
+        if (c > 0) {
+          tmem_ld32(tA + cc, v);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < D; cc += 32) {
-          uint32_t v[32];
-          if (c > 0) {
-            tmem_ld32(tA + cc, v);
-            tmem_wait_ld();
-          } else {
+          for (int t = 0; t < 32; ++t) v[t] = 0u;
+        }
+        if (key_ok) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
 #pragma unroll
-            for (int t = 0; t < 32; ++t) v[t] = 0u;
-          }
-          if (key_ok) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              uint4 w;
-              w.x = pack2<kFp16>(__uint_as_float(v[8 * t + 0]) * f, __uint_as_float(v[8 * t + 1]) * f);
-              w.y = pack2<kFp16>(__uint_as_float(v[8 * t + 2]) * f, __uint_as_float(v[8 * t + 3]) * f);
-              w.z = pack2<kFp16>(__uint_as_float(v[8 * t + 4]) * f, __uint_as_float(v[8 * t + 5]) * f);
-              w.w = pack2<kFp16>(__uint_as_float(v[8 * t + 6]) * f, __uint_as_float(v[8 * t + 7]) * f);
-              d4[t] = w;
-            }
+          for (int t = 0; t < 4; ++t) {
+            uint4 wv;
+            wv.x = pack2<kFp16>(__uint_as_float(v[8 * t + 0]) * f, __uint_as_float(v[8 * t + 1]) * f);
+            wv.y = pack2<kFp16>(__uint_as_float(v[8 * t + 2]) * f, __uint_as_float(v[8 * t + 3]) * f);
+            wv.z = pack2<kFp16>(__uint_as_float(v[8 * t + 4]) * f, __uint_as_float(v[8 * t + 5]) * f);
+            wv.w = pack2<kFp16>(__uint_as_float(v[8 * t + 6]) * f, __uint_as_float(v[8 * t + 7]) * f);
+            d4[t] = wv;
           }
         }
       }
     }
   } else {
-    // ------------------------------------------------------------------ dQ drain group (warps 4-7)
+    // ------------------------------------------------------------------ dQ drain group (warps 8-11)
     const int wq = warp & 3;
     const int r = wq * 32 + lane;                   // query row within the tile == TMEM lane
     const uint32_t tQ = tmem + C::tDQ + (static_cast<uint32_t>(wq * 32) << 16);
@@ -428,7 +458,7 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kBwdMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -442,7 +472,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.T);
-  kern<<<grid, 320, C::kSmem, s>>>(tq, tk, tv, tdo, a);
+  kern<<<grid, kBwdThreads, C::kSmem, s>>>(tq, tk, tv, tdo, a);
   return cudaGetLastError();
 }
 
