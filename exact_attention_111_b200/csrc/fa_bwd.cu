@@ -15,9 +15,9 @@
 //             partial of each step is added into the fp32 accumulator;
 //   bwd_post  dQ = 16-bit(scale * accumulator).
 //
-// bwd_main roles (448 threads): warps 0-7 two compute groups, one key row per thread (TMEM
-// lanes), each group owning half of the query columns; warps 8-11 drain dQ partials (one
-// query row per thread); warp 12 TMA producer; warp 13 MMA issuer.
+// bwd_main roles (320 threads): warps 0-7 two compute groups, one key row per thread (TMEM
+// lanes), each group owning half of the query columns and draining half of each dQ partial;
+// warp 8 TMA producer; warp 9 MMA issuer.
 // Tensor memory: Sᵀ/Pᵀ [0,128) (Pᵀ as 16-bit over the first 64 columns), dPᵀ [128,256),
 // dV and dK after them; dQ shares the dPᵀ columns when d = 128 and has its own for d = 64.
 // Per query tile, the MMAs: Sᵀ = K Q_iᵀ, dPᵀ = V dO_iᵀ, dV += Pᵀ dO_i (Pᵀ from TMEM),
@@ -120,9 +120,9 @@ struct BwdCfg {
   static constexpr bool kDqSharesDp = (D == 128);
 };
 
-constexpr int kBwdThreads = 448;   // 2 compute groups, dQ drain group, producer, MMA
-constexpr int kBwdLoadWarp = 12;
-constexpr int kBwdMmaWarp = 13;
+constexpr int kBwdThreads = 320;   // 2 compute groups (8 warps), producer, MMA issuer
+constexpr int kBwdLoadWarp = 8;
+constexpr int kBwdMmaWarp = 9;
 
 struct BwdBars {
   uint64_t kv_full;
@@ -149,8 +149,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   BwdBars& sh = *reinterpret_cast<BwdBars*>(smem + C::oBAR);
   const int warp = warp_id(), lane = lane_id();
-  const int bh = blockIdx.x % a.BH;
-  const int j = blockIdx.x / a.BH;                 // key tile; j = 0 first (heaviest under causal)
+  // CTAs resident together share a few heads, so those heads' Q / dO tiles and fp32 dQ
+  // accumulator rows stay in L2 (ordering by key tile across all heads thrashed L2); within
+  // a group, key tile 0 (the heaviest under causal masking) goes first.
+  int bh, j;
+  cta_order(blockIdx.x, a.BH, a.T, a.group_heads, bh, j);
   const DevStatus st{a.status, a.timeout_ns};
   volatile int* abort_flag = &sh.abort_flag;
   const bool aligned = (smem_addr(smem) & 1023u) == 0;
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sh.p_full, 256);
     mbar_init(&sh.ds_full, 256);
     mbar_init(&sh.dq_full, 1);
-    mbar_init(&sh.dq_empty, 128);
+    mbar_init(&sh.dq_empty, 256);
     mbar_init(&sh.mma_done, 1);
     sh.abort_flag = aligned ? 0 : 1;
     if (!aligned) atomicCAS(a.status, 0, kDevBadState);
@@ -313,21 +316,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait_drain(&sh.mma_done, 0, st);
     }
     __syncwarp();
-  } else if (warp < 8) {
+  } else {
     // ------------------------------------------------------------------ key-row compute groups
     // Group g (warps 4g..4g+3) owns query columns [64g, 64g+64) of every Sᵀ / dPᵀ tile; each
     // thread owns one key row (TMEM lane).  P stays in registers between the two phases.
+    // The groups also drain each dQ partial (query rows on TMEM lanes, half the columns each)
+    // right after the next P phase: the columns are released as soon as they are read, and
+    // the fp32 atomics follow from registers.
     const int g = warp >> 2;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;                   // key row within the tile == TMEM lane
     const int key = j * kTile + r;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + C::tS + lane_off, tDP = tmem + C::tDP + lane_off;
+    constexpr int kHalfD = D / 2;                   // dQ columns drained by each group
+    const uint32_t tQ = tmem + C::tDQ + lane_off + kHalfD * g;
     const float sl2 = a.scale_log2;
     const bool key_ok = key < a.N;
     uint8_t* ds_row = smem + C::oDS + g * C::kPanelBytes + r * 128;
     int c = 0;
     bool ok = true;
+    int i_prev = -1;
+    // dQ partial of query tile ip (the cq-th kept one), columns [kHalfD*g, kHalfD*(g+1)),
+    // -> fp32 accumulator
+    auto drain = [&](int ip, int cq) -> bool {
+      if (!mbar_wait(&sh.dq_full, cq & 1, abort_flag, st)) return false;
+      tc_fence_after();
+      uint32_t v[kHalfD];
+#pragma unroll
+      for (int cc = 0; cc < kHalfD; cc += 32) tmem_ld32(tQ + cc, *reinterpret_cast<uint32_t(*)[32]>(&v[cc]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&sh.dq_empty);
+      const int row = ip * kTile + r;               // query row == TMEM lane of the dQ tile
+      if (row < a.N) {
+        float4* dst = reinterpret_cast<float4*>(a.dq_acc + ((size_t)bh * a.N + row) * D + kHalfD * g);
+#pragma unroll
+        for (int t = 0; t < kHalfD / 4; ++t)
+          atomicAdd(dst + t, make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
+                                         __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3])));
+      }
+      return true;
+    };
     if (any) {
       for (int i = i_first; i < a.T; i = next_kept(i + 1, j, a.T, a.causal, a.blockmask), ++c) {
         const int s = c % C::kStages;
@@ -360,9 +390,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sh.p_full);
+        // dQ of the previous query tile (its completion also frees the dSᵀ buffer)
+        if (c > 0) {
+          ok = drain(i_prev, c - 1);
+          if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+        }
         // Phase B: dSᵀ = Pᵀ o (dPᵀ - D), 16-bit, into this group's shared-memory panel
-        ok = mbar_wait(&sh.dp_full, c & 1, abort_flag, st) &&
-             (c == 0 || mbar_wait(&sh.dq_full, (c - 1) & 1, abort_flag, st));   // dSᵀ buffer free
+        ok = mbar_wait(&sh.dp_full, c & 1, abort_flag, st);
         if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
@@ -389,7 +423,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(&sh.ds_full);
+        i_prev = i;
       }
+      if (ok && c > 0) ok = drain(i_prev, c - 1);
     }
     // Epilogue: group 0 writes dV, group 1 writes scale * dK, one key row per thread.
     if (ok) ok = mbar_wait(&sh.mma_done, 0, abort_flag, st);
@@ -422,36 +458,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             d4[t] = wv;
           }
         }
-      }
-    }
-  } else {
-    // ------------------------------------------------------------------ dQ drain group (warps 8-11)
-    const int wq = warp & 3;
-    const int r = wq * 32 + lane;                   // query row within the tile == TMEM lane
-    const uint32_t tQ = tmem + C::tDQ + (static_cast<uint32_t>(wq * 32) << 16);
-    int c = 0;
-    if (any) {
-      for (int i = i_first; i < a.T; i = next_kept(i + 1, j, a.T, a.causal, a.blockmask), ++c) {
-        bool ok = mbar_wait(&sh.dq_full, c & 1, abort_flag, st);
-        if (__any_sync(0xffffffffu, !ok)) break;
-        tc_fence_after();
-        const int row = i * kTile + r;
-        float* dst = a.dq_acc + ((size_t)bh * a.N + row) * D;
-#pragma unroll
-        for (int cc = 0; cc < D; cc += 32) {
-          uint32_t v[32];
-          tmem_ld32(tQ + cc, v);
-          tmem_wait_ld();
-          if (row < a.N) {
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-              atomicAdd(reinterpret_cast<float4*>(dst + cc) + t,
-                        make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
-                                    __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3])));
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&sh.dq_empty);
       }
     }
   }

@@ -68,9 +68,11 @@ __global__ void __launch_bounds__(320, 1)
   int* list = reinterpret_cast<int*>(sV + C::kStages * C::kTileBytes);  // T entries
 
   const int warp = warp_id(), lane = lane_id();
-  const int bh = blockIdx.x % a.BH;
-  int ui = blockIdx.x / a.BH;
-  if (a.causal) ui = a.n_units - 1 - ui;                  // heaviest query tiles first
+  // CTAs resident together work on a few heads (their K/V tiles then come from L2), and
+  // within that group the heaviest query units run first (causal: the last ones).
+  int bh, ui;
+  cta_order(blockIdx.x, a.BH, a.n_units, a.group_heads, bh, ui);
+  if (a.causal) ui = a.n_units - 1 - ui;
   const int qt0 = 2 * ui;
   const DevStatus st{a.status, a.timeout_ns};
   volatile int* abort_flag = &sh.abort_flag;
@@ -165,34 +167,32 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t idesc_s = idesc_f16(128, 128, kFp16, false, false);
       const uint32_t idesc_pv = idesc_f16(128, D, kFp16, false, true);
       const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
-      int npv[2] = {0, 0};
+      int npv0 = 0, npv1 = 0;                     // PV products issued per query tile
       for (int u = 0; u <= nu && ok; ++u) {
         const int ep = (u > 0) ? list[u - 1] : 0;
         const int ec = (u < nu) ? list[u] : 0;
         const int sp = (u + C::kStages - 1) % C::kStages;
         const int sc = u % C::kStages;
         bool v_ready = false, k_ready = false;
-        for (int q = 0; q < 2 && ok; ++q) {
+        // For query tile q: O_q += P_q V(u-1) if it kept tile u-1, then S_q = Q_q K(u)ᵀ if it keeps u.
+        auto step = [&](int q, int& npv) -> bool {
           if (u > 0 && ((ep >> (16 + q)) & 1)) {
             if (!v_ready) {
-              ok = mbar_wait(&sh.v_full[sp], ((u - 1) / C::kStages) & 1, abort_flag, st);
-              if (!ok) break;
+              if (!mbar_wait(&sh.v_full[sp], ((u - 1) / C::kStages) & 1, abort_flag, st)) return false;
               v_ready = true;
             }
-            ok = mbar_wait(&sh.p_full[q], npv[q] & 1, abort_flag, st);
-            if (!ok) break;
+            if (!mbar_wait(&sh.p_full[q], npv & 1, abort_flag, st)) return false;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk) {
               const uint64_t bdesc = smem_desc_sw128(aV + sp * C::kTileBytes + kk * 2048, C::kPanelBytes, 1024);
-              mma_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8, bdesc, idesc_pv, (npv[q] > 0 || kk > 0) ? 1u : 0u);
+              mma_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8, bdesc, idesc_pv, (npv > 0 || kk > 0) ? 1u : 0u);
             }
-            ++npv[q];
+            ++npv;
           }
           if (u < nu && ((ec >> (16 + q)) & 1)) {
             if (!k_ready) {
-              ok = mbar_wait(&sh.k_full[sc], (u / C::kStages) & 1, abort_flag, st);
-              if (!ok) break;
+              if (!mbar_wait(&sh.k_full[sc], (u / C::kStages) & 1, abort_flag, st)) return false;
               tc_fence_after();
               k_ready = true;
             }
@@ -207,7 +207,9 @@ __global__ void __launch_bounds__(320, 1)
             if (a.visit != nullptr)
               atomicAdd(&a.visit[((size_t)bh * a.T + (qt0 + q)) * a.T + (ec & 0xFFFF)], 1);
           }
-        }
+          return true;
+        };
+        ok = step(0, npv0) && step(1, npv1);
         if (u > 0 && ok) tc_commit(&sh.kv_empty[sp]);
       }
       if (ok) {
@@ -269,16 +271,22 @@ __global__ void __launch_bounds__(320, 1)
       }
       const float mneg = (m == -INFINITY) ? 0.f : -m;
       float sum0 = 0.f, sum1 = 0.f;
-      uint32_t pk[64];
+      // P in two halves of 64 keys, each stored to TMEM as soon as it is packed.
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2(fmaf(s[2 * i], sl2, mneg));
-        const float p1 = ex2(fmaf(s[2 * i + 1], sl2, mneg));
-        sum0 += p0;
-        sum1 += p1;
-        pk[i] = pack2<kFp16>(p0, p1);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2(fmaf(s[64 * h + 2 * i], sl2, mneg));
+          const float p1 = ex2(fmaf(s[64 * h + 2 * i + 1], sl2, mneg));
+          sum0 += p0;
+          sum1 += p1;
+          pk[i] = pack2<kFp16>(p0, p1);
+        }
+        tmem_st32(tS + 32 * h, pk);
       }
       l = l * alpha + (sum0 + sum1);
+      // O <- alpha O for the rows whose max grew (O holds every earlier PV product: see above)
       if (__any_sync(0xffffffffu, resc)) {
         const float f = resc ? alpha : 1.f;
 #pragma unroll
@@ -291,8 +299,6 @@ __global__ void __launch_bounds__(320, 1)
           tmem_st32(tO + cc, o);
         }
       }
-      tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sh.p_full[q]);

@@ -158,6 +158,7 @@ int fa_fwd_ex(const fa_fwd_args* p) {
   a.BH = BH;
   a.T = T;
   a.n_units = (T + 1) / 2;
+  a.group_heads = group_heads_for(BH, a.n_units);
   a.causal = x.causal != 0;
   a.o_fp32 = x.o_fp32 != 0;
   a.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
@@ -217,6 +218,7 @@ int fa_bwd_ex(const fa_bwd_args* p) {
   b.delta = delta; b.lse2 = lse2; b.dq_acc = dq_acc; b.dk = x.dk; b.dv = x.dv;
   b.blockmask = x.blockmask; b.visit = x.visit_log; b.status = status; b.timeout_ns = kWaitLimitNs;
   b.N = x.N; b.Np = Np; b.BH = BH; b.T = T; b.causal = x.causal != 0;
+  b.group_heads = group_heads_for(BH, T);
   b.scale = x.scale;
   b.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
   if (x.main_start_event && cudaEventRecord(static_cast<cudaEvent_t>(x.main_start_event), s) != cudaSuccess)

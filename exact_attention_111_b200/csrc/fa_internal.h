@@ -22,6 +22,7 @@ struct FwdArgs {
   int* status;              // device status word
   unsigned long long timeout_ns;
   int N, BH, T, n_units;    // n_units = ceil(T / 2): one CTA covers two 128-row query tiles
+  int group_heads;          // CTAs are ordered in groups of this many heads (see cta_order)
   int causal, o_fp32;
   float scale_log2;         // scale * log2(e)
 };
@@ -47,6 +48,7 @@ struct BwdArgs {
   int* status;
   unsigned long long timeout_ns;
   int N, Np, BH, T;
+  int group_heads;          // CTAs are ordered in groups of this many heads (see cta_order)
   int causal;
   float scale;              // multiplies dK (dQ is scaled in the post pass)
   float scale_log2;
@@ -68,5 +70,28 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 cudaError_t launch_bwd_post(const BwdPostArgs& a, bool fp16, cudaStream_t s);
 
 int* device_status_word();  // address of the per-process device status word
+
+// Heads per CTA-ordering group: about two waves of CTAs (148 SMs, one CTA each) per group, so
+// the heads a wave works on keep their tiles in L2 while each group still runs its heaviest
+// tiles first.
+inline int group_heads_for(int BH, int tiles_per_head) {
+  int g = (2 * 148 + tiles_per_head - 1) / tiles_per_head;
+  if (g < 1) g = 1;
+  if (g > BH) g = BH;
+  return g;
+}
+
+#ifdef __CUDACC__
+// CTA index -> (head, tile slot): heads in groups of G, tile slot outermost inside a group,
+// so slot 0 of every head in the group is scheduled before slot 1, and so on.
+__device__ __forceinline__ void cta_order(int idx, int BH, int tiles, int G, int& bh, int& slot) {
+  const int per = G * tiles;
+  const int grp = idx / per;
+  const int r = idx - grp * per;
+  const int heads_here = min(G, BH - grp * G);
+  slot = r / heads_here;
+  bh = grp * G + (r - slot * heads_here);
+}
+#endif
 
 }  // namespace fa
