@@ -132,12 +132,24 @@ struct BwdBars {
   int abort_flag;
 };
 
-// Next query tile at or after i that the key tile j keeps (T when none).
-__device__ __forceinline__ int next_kept(int i, int j, int T, int causal, const uint8_t* mask) {
-  if (causal && i < j) i = j;
-  if (mask != nullptr)
-    while (i < T && __ldg(mask + (size_t)i * T + j) == 0) ++i;
-  return i;
+// Query tiles are visited in the rotated order i = (j + k) mod T, k = 0, 1, ...: every key
+// tile starts at its own diagonal, so the CTAs of one head add their dQ partials into
+// different accumulator rows at any moment instead of all into the same ones.  Under causal
+// masking this is the natural order j, j+1, ..., T-1 (the wrapped part is all masked).
+__device__ __forceinline__ int rot_tile(int k, int j, int T) {
+  const int i = j + k;
+  return i < T ? i : i - T;
+}
+
+// Next step k' >= k whose query tile the key tile j keeps (T when none).
+__device__ __forceinline__ int next_kept(int k, int j, int T, int causal, const uint8_t* mask) {
+  for (; k < T; ++k) {
+    const int i = rot_tile(k, j, T);
+    if (causal && i < j) continue;
+    if (mask != nullptr && __ldg(mask + (size_t)i * T + j) == 0) continue;
+    break;
+  }
+  return k;
 }
 
 template <int D, bool kFp16>
@@ -183,8 +195,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
-  const int i_first = next_kept(0, j, a.T, a.causal, a.blockmask);
-  const bool any = aligned && i_first < a.T;
+  const int k_first = next_kept(0, j, a.T, a.causal, a.blockmask);
+  const bool any = aligned && k_first < a.T;
 
   if (warp == kBwdLoadWarp) {
     // ------------------------------------------------------------------ TMA producer
@@ -199,7 +211,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_3d(smem + C::oV + p * C::kPanelBytes, &tm_v, &sh.kv_full, p * 64, j * kTile, bh);
       }
       int c = 0;
-      for (int i = i_first; i < a.T; i = next_kept(i + 1, j, a.T, a.causal, a.blockmask), ++c) {
+      for (int k = k_first; k < a.T; k = next_kept(k + 1, j, a.T, a.causal, a.blockmask), ++c) {
+        const int i = rot_tile(k, j, a.T);
         const int s = c % C::kStages;
         if (c >= C::kStages && !mbar_wait(&sh.q_empty[s], ((c / C::kStages) - 1) & 1, abort_flag, st)) break;
         mbar_arrive_expect_tx(&sh.q_full[s], 2 * C::kTileBytes + 2 * kTile * 4);
@@ -259,12 +272,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (ok) {
         tc_fence_after();
         issue_s(0);
-        if (a.visit != nullptr) atomicAdd(&a.visit[((size_t)bh * a.T + i_first) * a.T + j], 1);
+        if (a.visit != nullptr) atomicAdd(&a.visit[((size_t)bh * a.T + rot_tile(k_first, j, a.T)) * a.T + j], 1);
         issue_dp(0);
-        for (int i = i_first; i < a.T; ++c) {
+        for (int k = k_first; k < a.T; ++c) {
           const int s = c % C::kStages;
-          const int i_next = next_kept(i + 1, j, a.T, a.causal, a.blockmask);
-          const bool more = i_next < a.T;
+          const int k_next = next_kept(k + 1, j, a.T, a.causal, a.blockmask);
+          const bool more = k_next < a.T;
+          const int i_next = more ? rot_tile(k_next, j, a.T) : 0;
           const uint32_t qb = aQ + s * C::kTileBytes, dob = aDO + s * C::kTileBytes;
           // dV += Pᵀ dO(c)   (Pᵀ read from tensor memory)
           if (!(ok = mbar_wait(&sh.p_full, c & 1, abort_flag, st))) break;
@@ -309,7 +323,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             issue_dp((c + 1) % C::kStages);
           }
-          i = i_next;
+          k = k_next;
         }
       }
       tc_commit(&sh.mma_done);
@@ -338,28 +352,50 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     int i_prev = -1;
     // dQ partial of query tile ip (the cq-th kept one), columns [kHalfD*g, kHalfD*(g+1)),
-    // -> fp32 accumulator
+    // -> fp32 accumulator.  The TMEM columns are released as soon as they are read.
     auto drain = [&](int ip, int cq) -> bool {
-      if (!mbar_wait(&sh.dq_full, cq & 1, abort_flag, st)) return false;
+      const bool got = mbar_wait(&sh.dq_full, cq & 1, abort_flag, st);
+      if (!__all_sync(0xffffffffu, got)) return false;   // warp-uniform before warp-collective loads
       tc_fence_after();
       uint32_t v[kHalfD];
 #pragma unroll
       for (int cc = 0; cc < kHalfD; cc += 32) tmem_ld32(tQ + cc, *reinterpret_cast<uint32_t(*)[32]>(&v[cc]));
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&sh.dq_empty);
-      const int row = ip * kTile + r;               // query row == TMEM lane of the dQ tile
-      if (row < a.N) {
-        float4* dst = reinterpret_cast<float4*>(a.dq_acc + ((size_t)bh * a.N + row) * D + kHalfD * g);
+      mbar_arrive(&sh.dq_empty);                    // TMEM columns free for the next MMA
+      // Lanes 2m and 2m+1 hold query rows R and R+1.  They swap one float4 per pair of
+      // float4 columns so that each vector atomic of the pair covers one whole 32-byte
+      // sector of one row: first (R, 2c | 2c+1), then (R+1, 2c | 2c+1).  L2 reduction
+      // throughput is counted in sectors, so this halves the sectors per dQ partial.
+      const bool odd = (lane & 1) != 0;
+      const int row_own = ip * kTile + r;           // query row == TMEM lane of the dQ tile
+      const int row_even = row_own - (odd ? 1 : 0);
+      float* base_even = a.dq_acc + ((size_t)bh * a.N + row_even) * D + kHalfD * g;
+      const bool ok0 = row_even < a.N, ok1 = row_even + 1 < a.N;
 #pragma unroll
-        for (int t = 0; t < kHalfD / 4; ++t)
-          atomicAdd(dst + t, make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
-                                         __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3])));
+      for (int c2 = 0; c2 < kHalfD / 8; ++c2) {
+        const float4 lo = make_float4(__uint_as_float(v[8 * c2 + 0]), __uint_as_float(v[8 * c2 + 1]),
+                                      __uint_as_float(v[8 * c2 + 2]), __uint_as_float(v[8 * c2 + 3]));
+        const float4 hi = make_float4(__uint_as_float(v[8 * c2 + 4]), __uint_as_float(v[8 * c2 + 5]),
+                                      __uint_as_float(v[8 * c2 + 6]), __uint_as_float(v[8 * c2 + 7]));
+        const float4 send = odd ? lo : hi;          // even sends its upper half, odd its lower
+        float4 recv;
+        recv.x = __shfl_xor_sync(0xffffffffu, send.x, 1);
+        recv.y = __shfl_xor_sync(0xffffffffu, send.y, 1);
+        recv.z = __shfl_xor_sync(0xffffffffu, send.z, 1);
+        recv.w = __shfl_xor_sync(0xffffffffu, send.w, 1);
+        // first write: row R, float4 index 2*c2 (even, own lo) | 2*c2+1 (odd, received hi)
+        // second write: row R+1, float4 index 2*c2 (even, received lo) | 2*c2+1 (odd, own hi)
+        float4* p0 = reinterpret_cast<float4*>(base_even) + 2 * c2 + (odd ? 1 : 0);
+        float4* p1 = reinterpret_cast<float4*>(base_even + D) + 2 * c2 + (odd ? 1 : 0);
+        if (ok0) atomicAdd(p0, odd ? recv : lo);
+        if (ok1) atomicAdd(p1, odd ? hi : recv);
       }
       return true;
     };
     if (any) {
-      for (int i = i_first; i < a.T; i = next_kept(i + 1, j, a.T, a.causal, a.blockmask), ++c) {
+      for (int k = k_first; k < a.T; k = next_kept(k + 1, j, a.T, a.causal, a.blockmask), ++c) {
+        const int i = rot_tile(k, j, a.T);
         const int s = c % C::kStages;
         ok = mbar_wait(&sh.q_full[s], (c / C::kStages) & 1, abort_flag, st) &&
              mbar_wait(&sh.s_full, c & 1, abort_flag, st);
