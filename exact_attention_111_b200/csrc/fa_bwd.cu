@@ -18,7 +18,7 @@
 // bwd_main roles (320 threads): warps 0-7 two compute groups, one key row per thread (TMEM
 // lanes), each group owning half of the query columns and draining half of each dQ partial;
 // warp 8 TMA producer; warp 9 MMA issuer.
-// Tensor memory: Sᵀ/Pᵀ [0,128) (Pᵀ as 16-bit over the first 64 columns), dPᵀ [128,256),
+// Tensor memory: Sᵀ/Pᵀ [0,128) (Pᵀ as 16-bit over columns [0,32) and [64,96)), dPᵀ [128,256),
 // dV and dK after them; dQ shares the dPᵀ columns when d = 128 and has its own for d = 64.
 // Per query tile, the MMAs: Sᵀ = K Q_iᵀ, dPᵀ = V dO_iᵀ, dV += Pᵀ dO_i (Pᵀ from TMEM),
 // dK += dSᵀ Q_i, dQ_i = dS K, issued one tile ahead where TMEM allows (see the MMA role)
@@ -283,10 +283,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // dV += Pᵀ dO(c)   (Pᵀ read from tensor memory)
           if (!(ok = mbar_wait(&sh.p_full, c & 1, abort_flag, st))) break;
           tc_fence_after();
+          // Pᵀ query columns 16kk..16kk+15 sit in TMEM columns 64*(kk/4) + 8*(kk%4) (see the compute groups)
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + C::tDV, tmem + C::tS + kk * 8, smem_desc_sw128(dob + kk * 2048, C::kPanelBytes, 1024), id_kn,
-                   (c > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + C::tDV, tmem + C::tS + (kk >> 2) * 64 + (kk & 3) * 8,
+                   smem_desc_sw128(dob + kk * 2048, C::kPanelBytes, 1024), id_kn, (c > 0 || kk > 0) ? 1u : 0u);
           // Sᵀ(c+1)
           if (more) {
             const int s1 = (c + 1) % C::kStages;
@@ -361,6 +362,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < kHalfD; cc += 32) tmem_ld32(tQ + cc, *reinterpret_cast<uint32_t(*)[32]>(&v[cc]));
       tmem_wait_ld();
+#pragma unroll
+      for (int cc = 0; cc < kHalfD; cc += 32) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&v[cc]));
       tc_fence_before();
       mbar_arrive(&sh.dq_empty);                    // TMEM columns free for the next MMA
       // Lanes 2m and 2m+1 hold query rows R and R+1.  They swap one float4 per pair of
@@ -409,8 +412,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t sv[32];
-          tmem_ld32(tS + 64 * g + 32 * h, sv);
-          tmem_wait_ld();
+          tmem_ld32_sync(tS + 64 * g + 32 * h, sv);
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
             const int ql = 32 * h + 2 * t;          // column within this group's 64
@@ -422,7 +424,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             pk[16 * h + t] = pack2<kFp16>(p0, p1);
           }
         }
-        tmem_st32(tS + 32 * g, pk);
+        // Pᵀ of this group's 64 query columns, packed two per 32-bit column, goes over the
+        // first half of the group's own Sᵀ columns [64g, 64g+32): the other group may still be
+        // reading its Sᵀ columns, so neither group writes outside its own range.
+        tmem_st32(tS + 64 * g, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sh.p_full);
@@ -438,8 +443,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t dpv[32];
-          tmem_ld32(tDP + 64 * g + 32 * h, dpv);
-          tmem_wait_ld();
+          tmem_ld32_sync(tDP + 64 * g + 32 * h, dpv);
           uint32_t w[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
@@ -476,8 +480,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int cc = 0; cc < D; cc += 32) {
         uint32_t v[32];
         if (c > 0) {
-          tmem_ld32(tA + cc, v);
-          tmem_wait_ld();
+          tmem_ld32_sync(tA + cc, v);
         } else {
 #pragma unroll
           for (int t = 0; t < 32; ++t) v[t] = 0u;

@@ -248,6 +248,8 @@ __global__ void __launch_bounds__(320, 1)
       tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       tmem_wait_ld();
+#pragma unroll
+      for (int cq = 0; cq < 4; ++cq) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cq]));
       float s[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
@@ -292,8 +294,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int cc = 0; cc < D; cc += 32) {
           uint32_t o[32];
-          tmem_ld32(tO + cc, o);
-          tmem_wait_ld();
+          tmem_ld32_sync(tO + cc, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
           tmem_st32(tO + cc, o);
@@ -318,8 +319,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int cc = 0; cc < D; cc += 32) {
         uint32_t o[32];
         if (nq > 0) {
-          tmem_ld32(tO + cc, o);
-          tmem_wait_ld();
+          tmem_ld32_sync(tO + cc, o);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0u;

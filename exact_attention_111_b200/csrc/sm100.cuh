@@ -229,6 +229,28 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// tcgen05.ld writes its destination registers asynchronously: they hold the loaded values
+// only after tcgen05.wait::ld.  The compiler cannot see that, so arithmetic on the loaded
+// registers could be scheduled between the load and the wait.  After each wait, pass the
+// registers through an empty volatile asm that the compiler must assume rewrites them: every
+// later use then depends on it, and it is ordered after the (volatile) wait.
+__device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]));
+}
+__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
+  reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+  reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+}
+// Load 32 columns and wait for them (one warp-collective step).
+__device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_ld32(taddr, r);
+  tmem_wait_ld();
+  reg_fence32(r);
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------------------------
