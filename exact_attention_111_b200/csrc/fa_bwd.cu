@@ -156,7 +156,7 @@ template <int D, bool kFp16>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const BwdArgs a) {
+               const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   BwdBars& sh = *reinterpret_cast<BwdBars*>(smem + C::oBAR);
@@ -353,7 +353,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     int i_prev = -1;
     // dQ partial of query tile ip (the cq-th kept one), columns [kHalfD*g, kHalfD*(g+1)),
-    // -> fp32 accumulator.  The TMEM columns are released as soon as they are read.
+    // -> fp32 accumulator.  The group's dSᵀ panel (16 KB, free once dq_full says dK / dQ
+    // have read it) stages 32 columns at a time in the 128-byte-swizzled layout of the
+    // accumulator's TMA map; each warp stages its own 32 rows (4 KB) and its lane 0 issues a
+    // TMA tensor reduce-add for them, so the reduction runs on the TMA engine instead of as
+    // per-thread atomics, and only warp-level synchronisation is needed.
+    uint8_t* stage = smem + C::oDS + g * C::kPanelBytes + wq * 32 * 128;
     auto drain = [&](int ip, int cq) -> bool {
       const bool got = mbar_wait(&sh.dq_full, cq & 1, abort_flag, st);
       if (!__all_sync(0xffffffffu, got)) return false;   // warp-uniform before warp-collective loads
@@ -366,33 +371,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int cc = 0; cc < kHalfD; cc += 32) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&v[cc]));
       tc_fence_before();
       mbar_arrive(&sh.dq_empty);                    // TMEM columns free for the next MMA
-      // Lanes 2m and 2m+1 hold query rows R and R+1.  They swap one float4 per pair of
-      // float4 columns so that each vector atomic of the pair covers one whole 32-byte
-      // sector of one row: first (R, 2c | 2c+1), then (R+1, 2c | 2c+1).  L2 reduction
-      // throughput is counted in sectors, so this halves the sectors per dQ partial.
-      const bool odd = (lane & 1) != 0;
-      const int row_own = ip * kTile + r;           // query row == TMEM lane of the dQ tile
-      const int row_even = row_own - (odd ? 1 : 0);
-      float* base_even = a.dq_acc + ((size_t)bh * a.N + row_even) * D + kHalfD * g;
-      const bool ok0 = row_even < a.N, ok1 = row_even + 1 < a.N;
 #pragma unroll
-      for (int c2 = 0; c2 < kHalfD / 8; ++c2) {
-        const float4 lo = make_float4(__uint_as_float(v[8 * c2 + 0]), __uint_as_float(v[8 * c2 + 1]),
-                                      __uint_as_float(v[8 * c2 + 2]), __uint_as_float(v[8 * c2 + 3]));
-        const float4 hi = make_float4(__uint_as_float(v[8 * c2 + 4]), __uint_as_float(v[8 * c2 + 5]),
-                                      __uint_as_float(v[8 * c2 + 6]), __uint_as_float(v[8 * c2 + 7]));
-        const float4 send = odd ? lo : hi;          // even sends its upper half, odd its lower
-        float4 recv;
-        recv.x = __shfl_xor_sync(0xffffffffu, send.x, 1);
-        recv.y = __shfl_xor_sync(0xffffffffu, send.y, 1);
-        recv.z = __shfl_xor_sync(0xffffffffu, send.z, 1);
-        recv.w = __shfl_xor_sync(0xffffffffu, send.w, 1);
-        // first write: row R, float4 index 2*c2 (even, own lo) | 2*c2+1 (odd, received hi)
-        // second write: row R+1, float4 index 2*c2 (even, received lo) | 2*c2+1 (odd, own hi)
-        float4* p0 = reinterpret_cast<float4*>(base_even) + 2 * c2 + (odd ? 1 : 0);
-        float4* p1 = reinterpret_cast<float4*>(base_even + D) + 2 * c2 + (odd ? 1 : 0);
-        if (ok0) atomicAdd(p0, odd ? recv : lo);
-        if (ok1) atomicAdd(p1, odd ? hi : recv);
+      for (int rd = 0; rd < kHalfD / 32; ++rd) {
+        uint8_t* row_base = stage + lane * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const int phys = ch ^ (lane & 7);
+          *reinterpret_cast<uint4*>(row_base + phys * 16) =
+              make_uint4(v[32 * rd + 4 * ch], v[32 * rd + 4 * ch + 1], v[32 * rd + 4 * ch + 2], v[32 * rd + 4 * ch + 3]);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tm_dq, stage, kHalfD * g + 32 * rd, ip * kTile + wq * 32, bh);
+          bulk_commit();
+          bulk_wait_read_all();                     // staging rows may be overwritten again
+        }
+        __syncwarp();
       }
       return true;
     };
@@ -466,6 +461,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         i_prev = i;
       }
       if (ok && c > 0) ok = drain(i_prev, c - 1);
+      if (lane == 0) bulk_wait_all();
     }
     // Epilogue: group 0 writes dV, group 1 writes scale * dK, one key row per thread.
     if (ok) ok = mbar_wait(&sh.mma_done, 0, abort_flag, st);
@@ -511,13 +507,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 template <int D, bool kFp16>
 cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                         const BwdArgs& a, cudaStream_t s) {
+                         const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t s) {
   using C = BwdCfg<D>;
   auto kern = bwd_kernel<D, kFp16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.T);
-  kern<<<grid, kBwdThreads, C::kSmem, s>>>(tq, tk, tv, tdo, a);
+  kern<<<grid, kBwdThreads, C::kSmem, s>>>(tq, tk, tv, tdo, tdq, a);
   return cudaGetLastError();
 }
 
@@ -546,9 +542,10 @@ cudaError_t launch_bwd_pre(const BwdPreArgs& a, bool fp16, cudaStream_t s) {
 }
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const BwdArgs& a, int d, bool fp16, cudaStream_t s) {
-  if (d == 64) return fp16 ? launch_bwd_t<64, true>(tq, tk, tv, tdo, a, s) : launch_bwd_t<64, false>(tq, tk, tv, tdo, a, s);
-  return fp16 ? launch_bwd_t<128, true>(tq, tk, tv, tdo, a, s) : launch_bwd_t<128, false>(tq, tk, tv, tdo, a, s);
+                       const CUtensorMap& tdq, const BwdArgs& a, int d, bool fp16, cudaStream_t s) {
+  if (d == 64)
+    return fp16 ? launch_bwd_t<64, true>(tq, tk, tv, tdo, tdq, a, s) : launch_bwd_t<64, false>(tq, tk, tv, tdo, tdq, a, s);
+  return fp16 ? launch_bwd_t<128, true>(tq, tk, tv, tdo, tdq, a, s) : launch_bwd_t<128, false>(tq, tk, tv, tdo, tdq, a, s);
 }
 
 cudaError_t launch_bwd_post(const BwdPostArgs& a, bool fp16, cudaStream_t s) {

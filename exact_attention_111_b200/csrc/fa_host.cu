@@ -55,6 +55,19 @@ bool encode_qkv(CUtensorMap* m, const void* base, int BH, int N, int d, bool fp1
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 dQ accumulator [BH, N, d] as a 3-D TMA map with 32 x 32 x 1 boxes (32 columns = 128
+// bytes wide, 32 rows: one warp's rows), 128-byte swizzle, for tensor reduce-add from shared
+// memory; rows past N are skipped.
+bool encode_dqacc(CUtensorMap* m, const void* base, int BH, int N, int d) {
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)N * d * 4};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 int check_shape(int B, int H, int N, int d, float scale, int dtype) {
@@ -201,6 +214,8 @@ int fa_bwd_ex(const fa_bwd_args* p) {
     return FA_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(x.workspace);
   float* dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
+  CUtensorMap tdq;
+  if (!encode_dqacc(&tdq, dq_acc, BH, x.N, x.d)) return FA_ERR_CUDA;
   float* delta = reinterpret_cast<float*>(ws + w.delta);
   float* lse2 = reinterpret_cast<float*>(ws + w.lse2);
   cudaStream_t s = static_cast<cudaStream_t>(x.stream);
@@ -223,7 +238,7 @@ int fa_bwd_ex(const fa_bwd_args* p) {
   b.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
   if (x.main_start_event && cudaEventRecord(static_cast<cudaEvent_t>(x.main_start_event), s) != cudaSuccess)
     return FA_ERR_CUDA;
-  if (launch_bwd(tq, tk, tv, tdo, b, x.d, fp16, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd(tq, tk, tv, tdo, tdq, b, x.d, fp16, s) != cudaSuccess) return FA_ERR_CUDA;
   if (x.main_stop_event && cudaEventRecord(static_cast<cudaEvent_t>(x.main_stop_event), s) != cudaSuccess)
     return FA_ERR_CUDA;
 

@@ -66,7 +66,8 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        int d, bool fp16, cudaStream_t s);
 cudaError_t launch_bwd_pre(const BwdPreArgs& a, bool fp16, cudaStream_t s);
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdArgs& a, int d, bool fp16, cudaStream_t s);
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int d, bool fp16,
+                       cudaStream_t s);
 cudaError_t launch_bwd_post(const BwdPostArgs& a, bool fp16, cudaStream_t s);
 
 int* device_status_word();  // address of the per-process device status word
