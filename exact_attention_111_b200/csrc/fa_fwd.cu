@@ -260,9 +260,16 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < 128; ++i)
           if (i >= lim) s[i] = -INFINITY;
       }
-      float mx = s[0];
+      // Row max: eight independent chains of 3-input maxima (depth 10 instead of a 127-long
+      // dependent chain), then one combine.
+      float mxa[8];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      for (int k = 0; k < 8; ++k) mxa[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+      for (int i = 16; i < 128; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mxa[k] = max3f(mxa[k], s[i + 2 * k], s[i + 2 * k + 1]);
+      const float mx = max3f(max3f(mxa[0], mxa[1], mxa[2]), max3f(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
       const float mx2 = mx * sl2;
       float alpha = 1.f;
       bool resc = false;
@@ -272,21 +279,25 @@ __global__ void __launch_bounds__(320, 1)
         m = mx2;
       }
       const float mneg = (m == -INFINITY) ? 0.f : -m;
-      float sum0 = 0.f, sum1 = 0.f;
-      // P in two halves of 64 keys, each stored to TMEM as soon as it is packed.
+      const float2 sl2v = make_float2(sl2, sl2), mnegv = make_float2(mneg, mneg);
+      // P = 2^(s*scale*log2e - m) in pairs (packed fp32 FMA), row sum over four packed
+      // accumulators; P stored to TMEM in quarters of 32 keys as soon as each is packed.
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
+      for (int h = 0; h < 4; ++h) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(fmaf(s[64 * h + 2 * i], sl2, mneg));
-          const float p1 = ex2(fmaf(s[64 * h + 2 * i + 1], sl2, mneg));
-          sum0 += p0;
-          sum1 += p1;
-          pk[i] = pack2<kFp16>(p0, p1);
+        for (int i = 0; i < 16; ++i) {
+          const float2 t = fma2(make_float2(s[32 * h + 2 * i], s[32 * h + 2 * i + 1]), sl2v, mnegv);
+          const float2 p = make_float2(ex2(t.x), ex2(t.y));
+          acc[i & 3] = add2(acc[i & 3], p);
+          pk[i] = pack2<kFp16>(p.x, p.y);
         }
-        tmem_st32(tS + 32 * h, pk);
+        tmem_st16(tS + 16 * h, pk);
       }
+      const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+      const float2 a0123 = add2(a01, a23);
+      const float sum0 = a0123.x, sum1 = a0123.y;
       l = l * alpha + (sum0 + sum1);
       // O <- alpha O for the rows whose max grew (O holds every earlier PV product: see above)
       if (__any_sync(0xffffffffu, resc)) {
@@ -296,7 +307,11 @@ __global__ void __launch_bounds__(320, 1)
           uint32_t o[32];
           tmem_ld32_sync(tO + cc, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 r = mul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), make_float2(f, f));
+            o[i] = __float_as_uint(r.x);
+            o[i + 1] = __float_as_uint(r.y);
+          }
           tmem_st32(tO + cc, o);
         }
       }
