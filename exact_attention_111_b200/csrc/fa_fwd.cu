@@ -38,6 +38,8 @@ struct FwdCfg {
   static constexpr int kStages = (D == 64) ? 4 : 2;      // K/V ring depth
   static constexpr int kSmemTiles = 2 * kTileBytes + 2 * kStages * kTileBytes;
   static constexpr int kThreads = 320;
+  // exp2 pairs per 8 evaluated by polynomial on the FMA pipe instead of the SFU
+  static constexpr int kPolyOf8 = (D == 64) ? 2 : 0;
 };
 
 struct FwdShared {
@@ -289,7 +291,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float2 t = fma2(make_float2(s[32 * h + 2 * i], s[32 * h + 2 * i + 1]), sl2v, mnegv);
-          const float2 p = make_float2(ex2(t.x), ex2(t.y));
+          // kPolyOf8 of every 8 pairs go to the FMA-pipe polynomial, the rest to the SFU
+          const float2 p = (((16 * h + i) & 7) < C::kPolyOf8) ? exp2_poly2(t) : make_float2(ex2(t.x), ex2(t.y));
           acc[i & 3] = add2(acc[i & 3], p);
           pk[i] = pack2<kFp16>(p.x, p.y);
         }

@@ -366,6 +366,26 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return f2unpack(r);
 }
 
+// 2^x for a pair of x <= 0 on the FMA/ALU pipes, to take load off the special-function unit.
+// x = j + f with j = round(x) (added to the exponent field) and f in [-1/2, 1/2];
+// 2^f ~ 1 + c1 f + c2 f^2 + c3 f^3, max relative error 1.0e-4 (coefficients fitted by
+// exact_attention_111_b200/fit_exp2_poly.py).  x is clamped at -127, where the result is
+// exactly +0 (so -inf, a masked score, gives 0); x = 0 gives exactly 1.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;            // 1.5 * 2^23: adding it rounds to an integer
+  constexpr float c1 = 6.932829022e-01f, c2 = 2.422109544e-01f, c3 = 5.500892922e-02f;
+  const float2 xc = make_float2(fmaxf(x.x, -127.f), fmaxf(x.y, -127.f));
+  const float2 t = add2(xc, make_float2(kRound, kRound));      // low mantissa bits hold j
+  const float2 j = add2(t, make_float2(-kRound, -kRound));
+  const float2 f = fma2(j, make_float2(-1.f, -1.f), xc);        // exact
+  float2 p = fma2(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = fma2(p, f, make_float2(c1, c1));
+  p = fma2(p, f, make_float2(1.f, 1.f));
+  // p * 2^j: add j to the exponent field (t's low 9 bits shifted up are exactly j << 23)
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
