@@ -8,7 +8,7 @@
 //     dS = P o (dP - D),  dQ = scale * dS K,  dK = scale * dSᵀ Q.
 //
 // Three kernels on one stream:
-//   bwd_pre   D_i, LSE_i*log2(e) (padded to whole tiles), and a zeroed fp32 dQ accumulator;
+//   bwd_pre   -D_i and -LSE_i*log2(e) (padded to whole tiles), and a zeroed fp32 dQ accumulator;
 //   bwd_main  one CTA per (b, h, 128-key tile j): K_j, V_j stay in shared memory while the
 //             CTA walks the kept 128-row query tiles i (i >= j under causal masking, and
 //             blockmask[i][j] != 0); dK_j, dV_j accumulate in tensor memory, the dQ_i
@@ -68,13 +68,13 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreArgs a) {
 #pragma unroll
     for (int s = G / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s, G);
     if (g == 0 && active) {
-      a.delta[r] = acc;
-      float l2 = INFINITY;                     // padding rows and rows with no visible key
+      a.delta[r] = -acc;                       // stored negated: the main kernel adds it
+      float nl2 = -INFINITY;                   // padding rows and rows with no visible key: P = 0
       if (i < a.N) {
         const float lse = a.lse[(size_t)bh * a.N + i];
-        if (lse > -INFINITY) l2 = lse * kLog2e;
+        if (lse > -INFINITY) nl2 = -lse * kLog2e;
       }
-      a.lse2[r] = l2;
+      a.lse2[r] = nl2;                         // -LSE * log2(e)
     }
   }
 }
@@ -399,24 +399,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
              mbar_wait(&sh.s_full, c & 1, abort_flag, st);
         if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
         tc_fence_after();
-        const float* lse2 = reinterpret_cast<const float*>(smem + C::oLSE + s * kTile * 4) + 64 * g;
-        const float* dlt = reinterpret_cast<const float*>(smem + C::oDELTA + s * kTile * 4) + 64 * g;
+        // -LSE*log2(e) and -D of this group's 64 query columns (bulk-loaded with the stage)
+        const float* nlse2 = reinterpret_cast<const float*>(smem + C::oLSE + s * kTile * 4) + 64 * g;
+        const float* ndlt = reinterpret_cast<const float*>(smem + C::oDELTA + s * kTile * 4) + 64 * g;
         const bool diag = a.causal && (i == j);     // key r visible to query column q iff r <= q
-        // Phase A: Pᵀ = 2^(scale*log2e*Sᵀ - LSE*log2e), 16-bit, over Sᵀ in TMEM
+        // Phase A: Pᵀ = 2^(scale*log2e*Sᵀ - LSE*log2e), 16-bit, over Sᵀ in TMEM.  Both
+        // 32-column chunks are loaded before one wait; -LSE*log2e comes in float4s; the
+        // exponent argument is one packed fp32 FMA per pair.
         uint32_t pk[32];
+        {
+          uint32_t sv[64];
+          tmem_ld32(tS + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(tS + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_wait_ld();
+          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          const float4* nl4 = reinterpret_cast<const float4*>(nlse2);
+          const float2 sl2v = make_float2(sl2, sl2);
+          const bool any_mask = !key_ok || diag;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sv[32];
-          tmem_ld32_sync(tS + 64 * g + 32 * h, sv);
+          for (int t4 = 0; t4 < 16; ++t4) {            // 4 query columns per step
+            const float4 nl = nl4[t4];
 #pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            const int ql = 32 * h + 2 * t;          // column within this group's 64
-            const int q0 = 64 * g + ql;             // column within the tile
-            float p0 = ex2(fmaf(__uint_as_float(sv[2 * t]), sl2, -lse2[ql]));
-            float p1 = ex2(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, -lse2[ql + 1]));
-            if (!key_ok || (diag && r > q0)) p0 = 0.f;
-            if (!key_ok || (diag && r > q0 + 1)) p1 = 0.f;
-            pk[16 * h + t] = pack2<kFp16>(p0, p1);
+            for (int hh = 0; hh < 2; ++hh) {
+              const int t = 2 * t4 + hh;                // pair index: columns 2t, 2t+1 of the 64
+              const float2 x = fma2(make_float2(__uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1])), sl2v,
+                                    hh == 0 ? make_float2(nl.x, nl.y) : make_float2(nl.z, nl.w));
+              float2 p = make_float2(ex2(x.x), ex2(x.y));
+              if (any_mask) {
+                const int q0 = 64 * g + 2 * t;          // column within the tile
+                if (!key_ok || (diag && r > q0)) p.x = 0.f;
+                if (!key_ok || (diag && r > q0 + 1)) p.y = 0.f;
+              }
+              pk[t] = pack2<kFp16>(p.x, p.y);
+            }
           }
         }
         // Pᵀ of this group's 64 query columns, packed two per 32-bit column, goes over the
@@ -435,24 +451,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = mbar_wait(&sh.dp_full, c & 1, abort_flag, st);
         if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
         tc_fence_after();
+        {
+          uint32_t dpv[64];
+          tmem_ld32(tDP + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&dpv[0]));
+          tmem_ld32(tDP + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&dpv[32]));
+          tmem_wait_ld();
+          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dpv[0]));
+          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dpv[32]));
+          const float4* nd4 = reinterpret_cast<const float4*>(ndlt);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t dpv[32];
-          tmem_ld32_sync(tDP + 64 * g + 32 * h, dpv);
-          uint32_t w[16];
+          for (int h = 0; h < 2; ++h) {
+            uint32_t w[16];
 #pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            const int ql = 32 * h + 2 * t;
-            const float2 p = unpack2<kFp16>(pk[16 * h + t]);
-            const float ds0 = p.x * (__uint_as_float(dpv[2 * t]) - dlt[ql]);
-            const float ds1 = p.y * (__uint_as_float(dpv[2 * t + 1]) - dlt[ql + 1]);
-            w[t] = pack2<kFp16>(ds0, ds1);
-          }
-          // 64 bytes = four 16-byte chunks of this key row (128-byte swizzle)
+            for (int t4 = 0; t4 < 8; ++t4) {
+              const float4 nd = nd4[8 * h + t4];
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int chunk = (h * 4 + t) ^ (r & 7);
-            *reinterpret_cast<uint4*>(ds_row + chunk * 16) = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
+              for (int hh = 0; hh < 2; ++hh) {
+                const int t = 16 * h + 2 * t4 + hh;     // pair index within the group's 64 columns
+                const float2 p = unpack2<kFp16>(pk[t]);
+                const float2 dp = make_float2(__uint_as_float(dpv[2 * t]), __uint_as_float(dpv[2 * t + 1]));
+                const float2 ds = mul2(p, add2(dp, hh == 0 ? make_float2(nd.x, nd.y) : make_float2(nd.z, nd.w)));
+                w[2 * t4 + hh] = pack2<kFp16>(ds.x, ds.y);
+              }
+            }
+            // 64 bytes = four 16-byte chunks of this key row (128-byte swizzle)
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const int chunk = (h * 4 + t) ^ (r & 7);
+              *reinterpret_cast<uint4*>(ds_row + chunk * 16) = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
+            }
           }
         }
         fence_async_smem();

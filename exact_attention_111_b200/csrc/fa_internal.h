@@ -31,15 +31,15 @@ struct BwdPreArgs {
   const void* o;            // [BH, N, d]
   const void* dout;         // [BH, N, d]
   const float* lse;         // [BH, N]
-  float* delta;             // [BH, Np]  D_i = sum_c dO_ic O_ic (0 on padding rows)
-  float* lse2;              // [BH, Np]  LSE_i * log2(e) (+inf on padding / empty rows)
+  float* delta;             // [BH, Np]  -D_i = -sum_c dO_ic O_ic (0 on padding rows)
+  float* lse2;              // [BH, Np]  -LSE_i * log2(e) (-inf on padding / empty rows)
   float* dq_acc;            // [BH, N, d] fp32, zeroed here
   int N, Np, BH, d;
 };
 
 struct BwdArgs {
-  const float* delta;       // [BH, Np]
-  const float* lse2;        // [BH, Np]
+  const float* delta;       // [BH, Np]  -D
+  const float* lse2;        // [BH, Np]  -LSE * log2(e)
   float* dq_acc;            // [BH, N, d]
   void* dk;                 // [BH, N, d] 16-bit
   void* dv;                 // [BH, N, d] 16-bit
