@@ -115,7 +115,15 @@ struct BwdCfg {
   static constexpr int oLSE = oDS + kTile * kTile * 2;
   static constexpr int oDELTA = oLSE + kStages * kTile * 4;
   static constexpr int oBAR = oDELTA + kStages * kTile * 4;
-  static constexpr int kSmem = oBAR + 256;
+  // dQ staging for the TMA reduce: its own 32 KB at d = 64 (the reduce's shared-memory read
+  // then overlaps the next tile's work); at d = 128 shared memory is full and the dSᵀ panels
+  // are reused, so the read must finish before the next dSᵀ tile is stored.
+  static constexpr bool kOwnStaging = (D == 64);
+  static constexpr int oSTG = ((oBAR + 256 + 1023) / 1024) * 1024;
+  static constexpr int kSmem = kOwnStaging ? oSTG + 2 * kPanelBytes : oBAR + 256;
+  // exp2 pairs per 8 evaluated by the FMA-pipe polynomial in the P phase (measured: 2 of 8
+  // helps slightly at d = 64, any share is slower at d = 128)
+  static constexpr int kPolyOf8 = (D == 64) ? 2 : 0;
   static constexpr int tS = 0, tDP = 128, tDV = 256, tDK = 256 + D, tDQ = (D == 128) ? 128 : 384;
   static constexpr bool kDqSharesDp = (D == 128);
 };
@@ -358,7 +366,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // accumulator's TMA map; each warp stages its own 32 rows (4 KB) and its lane 0 issues a
     // TMA tensor reduce-add for them, so the reduction runs on the TMA engine instead of as
     // per-thread atomics, and only warp-level synchronisation is needed.
-    uint8_t* stage = smem + C::oDS + g * C::kPanelBytes + wq * 32 * 128;
+    uint8_t* stage = smem + (C::kOwnStaging ? C::oSTG : C::oDS) + g * C::kPanelBytes + wq * 32 * 128;
+    // After a drain, lane 0 of each warp has reduce operations in flight that still read
+    // `stage`; wait_stage_read() must run before `stage` (or, at d = 128, the dSᵀ panel it lives
+    // in) is written again.
+    auto wait_stage_read = [&]() {
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+    };
     auto drain = [&](int ip, int cq) -> bool {
       const bool got = mbar_wait(&sh.dq_full, cq & 1, abort_flag, st);
       if (!__all_sync(0xffffffffu, got)) return false;   // warp-uniform before warp-collective loads
@@ -373,6 +388,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(&sh.dq_empty);                    // TMEM columns free for the next MMA
 #pragma unroll
       for (int rd = 0; rd < kHalfD / 32; ++rd) {
+        wait_stage_read();                          // previous reduce finished reading `stage`
         uint8_t* row_base = stage + lane * 128;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
@@ -385,9 +401,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (lane == 0) {
           tma_reduce_add_3d(&tm_dq, stage, kHalfD * g + 32 * rd, ip * kTile + wq * 32, bh);
           bulk_commit();
-          bulk_wait_read_all();                     // staging rows may be overwritten again
         }
-        __syncwarp();
       }
       return true;
     };
@@ -425,7 +439,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               const int t = 2 * t4 + hh;                // pair index: columns 2t, 2t+1 of the 64
               const float2 x = fma2(make_float2(__uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1])), sl2v,
                                     hh == 0 ? make_float2(nl.x, nl.y) : make_float2(nl.z, nl.w));
-              float2 p = make_float2(ex2(x.x), ex2(x.y));
+              float2 p = ((t & 7) < C::kPolyOf8) ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
               if (any_mask) {
                 const int q0 = 64 * g + 2 * t;          // column within the tile
                 if (!key_ok || (diag && r > q0)) p.x = 0.f;
@@ -459,27 +473,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dpv[0]));
           reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dpv[32]));
           const float4* nd4 = reinterpret_cast<const float4*>(ndlt);
+          uint32_t w[32];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t w[16];
+          for (int t4 = 0; t4 < 16; ++t4) {
+            const float4 nd = nd4[t4];
 #pragma unroll
-            for (int t4 = 0; t4 < 8; ++t4) {
-              const float4 nd = nd4[8 * h + t4];
-#pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                const int t = 16 * h + 2 * t4 + hh;     // pair index within the group's 64 columns
-                const float2 p = unpack2<kFp16>(pk[t]);
-                const float2 dp = make_float2(__uint_as_float(dpv[2 * t]), __uint_as_float(dpv[2 * t + 1]));
-                const float2 ds = mul2(p, add2(dp, hh == 0 ? make_float2(nd.x, nd.y) : make_float2(nd.z, nd.w)));
-                w[2 * t4 + hh] = pack2<kFp16>(ds.x, ds.y);
-              }
+            for (int hh = 0; hh < 2; ++hh) {
+              const int t = 2 * t4 + hh;                // pair index within the group's 64 columns
+              const float2 p = unpack2<kFp16>(pk[t]);
+              const float2 dp = make_float2(__uint_as_float(dpv[2 * t]), __uint_as_float(dpv[2 * t + 1]));
+              const float2 ds = mul2(p, add2(dp, hh == 0 ? make_float2(nd.x, nd.y) : make_float2(nd.z, nd.w)));
+              w[t] = pack2<kFp16>(ds.x, ds.y);
             }
-            // 64 bytes = four 16-byte chunks of this key row (128-byte swizzle)
+          }
+          // at d = 128 the dQ staging lives in this panel: its reduce must have read it
+          if (!C::kOwnStaging) wait_stage_read();
+          // 128 bytes = eight 16-byte chunks of this key row (128-byte swizzle)
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const int chunk = (h * 4 + t) ^ (r & 7);
-              *reinterpret_cast<uint4*>(ds_row + chunk * 16) = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
-            }
+          for (int t = 0; t < 8; ++t) {
+            const int chunk = t ^ (r & 7);
+            *reinterpret_cast<uint4*>(ds_row + chunk * 16) = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
           }
         }
         fence_async_smem();
