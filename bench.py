@@ -326,30 +326,59 @@ def run_ours(args, w, world, rank, local):
     bmain_tflops = bwd_flops / (bmain_ms * 1e-3) / 1e12
 
     # ---------------------------------------------------------------- end to end (host buffers)
+    # Every step copies its inputs from pinned host memory and its results (O, LSE, dQ, dK, dV)
+    # back to pinned host memory.  Device buffers are double-buffered and three streams
+    # (host->device, compute, device->host) overlap step k+1's upload and step k-1's download
+    # with step k's kernels; the timed region spans the first upload to the last download.
     e2e_steps = max(3, min(args.steps, 20))
-    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in
-                (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    sets = []
+    for _ in range(2):
+        din = {n: torch.empty_like(t) for n, t in d.items()}
+        dout_ = {"o": torch.empty_like(o), "lse": torch.empty_like(lse), "dq": torch.empty_like(dq),
+                 "dk": torch.empty_like(dk), "dv": torch.empty_like(dv)}
+        sets.append((din, dout_))
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in sets[0][1].items()}
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_down = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        for n in host:
-            d[n].copy_(host[n], non_blocking=True)
-        step()
-        host_out["o"].copy_(o, non_blocking=True)
-        host_out["lse"].copy_(lse, non_blocking=True)
-        host_out["dq"].copy_(dq, non_blocking=True)
-        host_out["dk"].copy_(dk, non_blocking=True)
-        host_out["dv"].copy_(dv, non_blocking=True)
+    def e2e_run(nsteps, t0=None, t1=None):
+        if t0 is not None:
+            t0.record(s_up)
+        for k in range(nsteps):
+            b = k % 2
+            din, dres = sets[b]
+            if k >= 2:
+                s_up.wait_event(ev_comp[b])          # step k-2 finished reading these inputs
+            with torch.cuda.stream(s_up):
+                for n in host:
+                    din[n].copy_(host[n], non_blocking=True)
+            ev_up[b].record(s_up)
+            stream.wait_event(ev_up[b])
+            if k >= 2:
+                stream.wait_event(ev_down[b])        # step k-2's results are on the host
+            fa.fa_fwd(din["q"], din["k"], din["v"], dres["o"], dres["lse"], B, H, N, D, scale, w.causal, mask, stream)
+            fa.fa_bwd(din["q"], din["k"], din["v"], dres["o"], dres["lse"], din["dout"], dres["dq"], dres["dk"],
+                      dres["dv"], B, H, N, D, scale, w.causal, mask, ws, wsb, stream)
+            ev_comp[b].record(stream)
+            s_down.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_down):
+                for n, t in dres.items():
+                    host_out[n].copy_(t, non_blocking=True)
+            ev_down[b].record(s_down)
+        if t1 is not None:
+            s_down.wait_stream(s_up)
+            s_down.wait_stream(stream)
+            t1.record(s_down)
 
-    e2e_step()
+    e2e_run(2)
     torch.cuda.synchronize(dev)
     barrier(world)
     s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    t2.record(stream)
+    e2e_run(e2e_steps, s2, t2)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(s2.elapsed_time(t2), world)
     e2e_value = aggregate_tflops(world, step_flops, e2e_steps, e2e_ms)
