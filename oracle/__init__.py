@@ -5,6 +5,8 @@ from .attention import (  # noqa: F401
     attention_bwd_head,
     attention_fwd,
     attention_fwd_head,
+    attention_fwd_partial,
     attention_fwd_head_tiled,
+    lse_merge,
     softmax_rows,
 )

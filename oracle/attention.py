@@ -33,6 +33,11 @@ Readings of points the pages leave open (each listed in the design doc):
   * block mask: uint8 [T, T] over 128 x 128 tiles, shared by all heads; a zero tile drops
     every score in it ("核心方法 / Block-sparse 扩展": zero blocks are skipped).
   * a row with no visible key has O = 0, LSE = -inf and zero gradients.
+  * a slice of the keys (one split of a split-KV forward, or one GPU's shard of a
+    sequence-sharded one): key row j of the slice is key position key_offset + j, and
+    causal and the block mask use that position.  Results over disjoint slices combine
+    exactly by ``lse_merge`` (the online-softmax rescaling of "核心方法 / Tiling 与 online
+    softmax", applied once per slice).
 
 Also here, for the oracle's own self-test only: ``attention_fwd_head_tiled`` -- the
 blockwise online-softmax recurrence of "核心方法 / Tiling 与 online softmax" (running row
@@ -47,15 +52,20 @@ import numpy as np
 TILE = 128
 
 
-def _keep_matrix(N: int, causal: bool, blockmask, tile: int = TILE) -> np.ndarray | None:
-    """Boolean [N, N]: True where score (i, j) takes part in the softmax; None = all."""
+def _keep_matrix(N: int, causal: bool, blockmask, tile: int = TILE, Nk: int | None = None,
+                 key_offset: int = 0) -> np.ndarray | None:
+    """Boolean [N, Nk]: True where score (i, j) takes part in the softmax; None = all.
+
+    Key row j sits at position ``key_offset + j`` of the query sequence (0 and Nk = N for
+    self-attention); causal and the block mask compare positions, not row indices."""
+    Nk = N if Nk is None else Nk
     keep = None
+    pos = key_offset + np.arange(Nk)
     if causal:
-        keep = np.tri(N, N, 0, dtype=bool)  # j <= i
+        keep = pos[None, :] <= np.arange(N)[:, None]
     if blockmask is not None:
         bm = np.asarray(blockmask).astype(bool)
-        t = np.arange(N) // tile
-        bk = bm[t[:, None], t[None, :]]
+        bk = bm[(np.arange(N) // tile)[:, None], (pos // tile)[None, :]]
         keep = bk if keep is None else (keep & bk)
     return keep
 
@@ -73,21 +83,45 @@ def softmax_rows(S: np.ndarray):
 
 
 def attention_fwd_head(q, k, v, scale: float, causal: bool = False, blockmask=None,
-                       return_p: bool = False, tile: int = TILE):
-    """One head: q, k, v are [N, d] float64.  Returns (O [N, d], LSE [N]) (and P).
-    ``tile`` is the block-mask tile side (128 for the product; small in oracle self-tests)."""
+                       return_p: bool = False, tile: int = TILE, key_offset: int = 0):
+    """One head: q is [N, d], k and v are [Nk, d] float64 (Nk = N for self-attention).
+    Returns (O [N, d], LSE [N]) (and P).  ``tile`` is the block-mask tile side (128 for the
+    product; small in oracle self-tests); ``key_offset`` places key row 0 in the query
+    sequence (a slice of the keys: one split or one shard)."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
     N = q.shape[0]
     S = scale * (q @ k.T)
-    keep = _keep_matrix(N, causal, blockmask, tile)
+    keep = _keep_matrix(N, causal, blockmask, tile, k.shape[0], key_offset)
     if keep is not None:
         S = np.where(keep, S, -np.inf)
     P, _, _, lse = softmax_rows(S)
     O = P @ v
     if return_p:
         return O, lse, P
+    return O, lse
+
+
+def lse_merge(o_parts, lse_parts):
+    """Combine attention results computed over disjoint key subsets of the same rows.
+
+    o_parts [S, ..., d] are each normalised over their own keys with log-sum-exp
+    lse_parts [S, ...].  Over the union of the keys the row sum of exp is the sum of the
+    parts' sums, so LSE = ln sum_s exp(LSE_s) and O = sum_s exp(LSE_s - LSE) O_s -- the same
+    rescaling that merges two blocks' running (m, l) statistics in the online softmax
+    (FlashAttention-NeurIPS22 summary, "核心方法 / Tiling 与 online softmax").  Rows where
+    every part saw no key stay O = 0, LSE = -inf."""
+    o_parts = np.asarray(o_parts, np.float64)
+    lse_parts = np.asarray(lse_parts, np.float64)
+    m = lse_parts.max(axis=0)
+    m_ref = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lse_parts - m_ref[None])               # 0 for parts that saw no key
+    tot = w.sum(axis=0)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        lse = np.where(tot > 0, m_ref + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+        frac = np.where(tot[None] > 0, w / np.where(tot > 0, tot, 1.0)[None], 0.0)
+    O = (frac[..., None] * o_parts).sum(axis=0)
     return O, lse
 
 
@@ -182,3 +216,19 @@ def attention_bwd(q, k, v, dout, scale: float, causal: bool = False, blockmask=N
         dQ[b, h], dK[b, h], dV[b, h], O[b, h], L[b, h] = attention_bwd_head(
             q[b, h], k[b, h], v[b, h], dout[b, h], scale, causal, bm)
     return dQ, dK, dV, O, L
+
+
+def attention_fwd_partial(q, k, v, scale: float, causal: bool = False, blockmask=None,
+                          key_offset: int = 0, heads=None):
+    """q: [B, H, N, d]; k, v: [B, H, Nk, d], key row 0 at position ``key_offset``.
+    Attention of every query row over these keys only: (O [B,H,N,d], LSE [B,H,N]) as
+    float64; unevaluated heads are NaN."""
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    B, H, N, _ = q.shape
+    bm = None if blockmask is None else _as64(blockmask)
+    O = np.full(q.shape[:3] + (v.shape[3],), np.nan)
+    L = np.full((B, H, N), np.nan)
+    for b, h in (heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]):
+        O[b, h], L[b, h] = attention_fwd_head(q[b, h], k[b, h], v[b, h], scale, causal, bm,
+                                              key_offset=key_offset)
+    return O, L

@@ -15,7 +15,13 @@ broken copy) and raises AssertionError when a fact fails.  The facts:
   * analytic gradients agree with central finite differences of L = sum(dO o O);
   * D_i = sum_j P_ij dP_ij equals sum_c dO_ic O_ic;
   * fp64 torch scaled_dot_product_attention (+ autograd) agrees on small shapes;
-  * a hand-derived two-key example (tests/golden/closed_forms.json).
+  * a hand-derived two-key example (tests/golden/closed_forms.json);
+  * a slice of the keys placed at a key offset (one split or one shard) matches a
+    brute-force double loop over explicit query and key positions;
+  * merging the results of disjoint key slices reaches the direct formula over all keys,
+    and the merge has closed forms: one part is the identity, two equal parts add ln 2 to
+    LSE, a part that saw no key contributes nothing, and LSEs ln 1 and ln 3 weigh the parts
+    1/4 and 3/4 (also at LSE near 1000, where exp itself overflows).
 """
 
 from __future__ import annotations
@@ -236,3 +242,92 @@ def eval_ln(x):
 
 ALL_FWD_PINS = (pin_rows_sum_to_one, pin_shift_invariance, pin_constant_v,
                 pin_zero_query_closed_form, pin_causal_row0, pin_d_identity)
+
+
+def _brute_slice(q, k, v, scale, causal, bm, tile, key_offset):
+    """Pure-Python double loop: row i sees key row j iff position key_offset + j passes."""
+    N, Nk = len(q), len(k)
+    O = [[0.0] * len(v[0]) for _ in range(N)]
+    L = [-math.inf] * N
+    for i in range(N):
+        sc = []
+        for j in range(Nk):
+            pos = key_offset + j
+            if causal and pos > i:
+                continue
+            if bm is not None and not bm[i // tile][pos // tile]:
+                continue
+            sc.append((j, scale * sum(float(a) * float(b) for a, b in zip(q[i], k[j]))))
+        if not sc:
+            continue
+        m = max(x for _, x in sc)
+        tot = sum(math.exp(x - m) for _, x in sc)
+        L[i] = m + math.log(tot)
+        for j, x in sc:
+            w = math.exp(x - m) / tot
+            for c in range(len(v[0])):
+                O[i][c] += w * float(v[j][c])
+    return np.array(O), np.array(L)
+
+
+def pin_key_slice_brute_force(fwd):
+    r = _rng(11)
+    N, d, tile = 13, 3, 4
+    q = r.standard_normal((N, d))
+    bm = np.array([[1, 1, 0, 1], [0, 1, 1, 1], [1, 0, 1, 0], [1, 1, 1, 1]], np.uint8)
+    for key_offset, Nk in ((0, 13), (4, 5), (8, 5), (12, 1), (4, 9)):
+        k, v = r.standard_normal((2, Nk, d))
+        for causal in (False, True):
+            for mask in (None, bm):
+                O, lse = fwd(q, k, v, 0.7, causal, mask, tile=tile, key_offset=key_offset)
+                Ob, Lb = _brute_slice(q, k, v, 0.7, causal, mask, tile, key_offset)
+                fin = np.isfinite(Lb)
+                assert np.array_equal(np.isfinite(lse), fin), (key_offset, causal)
+                assert np.max(np.abs(lse[fin] - Lb[fin]), initial=0.0) < 1e-12, (key_offset, causal)
+                assert np.max(np.abs(O - Ob)) < 1e-12, (key_offset, causal)
+
+
+def pin_merge_partition(fwd, merge):
+    """Partials over a partition of the keys, merged, equal attention over all keys."""
+    r = _rng(12)
+    N, d, tile = 23, 5, 4
+    q, k, v = r.standard_normal((3, N, d))
+    bm = (r.random((6, 6)) < 0.6).astype(np.uint8)
+    bm[3, :] = 0                                   # tile row 3: no visible key at all
+    for cuts in ((0, 23), (0, 8, 23), (0, 4, 12, 16, 23), (0, 20, 23)):
+        for causal in (False, True):
+            for mask in (None, bm):
+                Of, Lf = fwd(q, k, v, 0.4, causal, mask, tile=tile)
+                parts = [fwd(q, k[a:b], v[a:b], 0.4, causal, mask, tile=tile, key_offset=a)
+                         for a, b in zip(cuts[:-1], cuts[1:])]
+                O, L = merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+                fin = np.isfinite(Lf)
+                assert np.array_equal(np.isfinite(L), fin), (cuts, causal)
+                assert np.max(np.abs(L[fin] - Lf[fin]), initial=0.0) < 1e-12, (cuts, causal)
+                assert np.max(np.abs(O - Of)) < 1e-12, (cuts, causal)
+
+
+def pin_merge_closed_forms(merge):
+    r = _rng(13)
+    o1, o2 = r.standard_normal((2, 6, 4))
+    l1 = r.standard_normal(6)
+    # one part: identity
+    O, L = merge(o1[None], l1[None])
+    assert np.max(np.abs(O - o1)) < 1e-15 and np.max(np.abs(L - l1)) < 1e-15
+    # two equal parts: same O, LSE + ln 2
+    O, L = merge(np.stack([o1, o1]), np.stack([l1, l1]))
+    assert np.max(np.abs(O - o1)) < 1e-14 and np.max(np.abs(L - (l1 + math.log(2.0)))) < 1e-14
+    # a part that saw no key (LSE = -inf) contributes nothing, whatever its O holds
+    ninf = np.full(6, -np.inf)
+    O, L = merge(np.stack([o1, o2]), np.stack([l1, ninf]))
+    assert np.max(np.abs(O - o1)) < 1e-15 and np.max(np.abs(L - l1)) < 1e-15
+    # no part saw a key: O = 0, LSE = -inf
+    O, L = merge(np.stack([o1, o2]), np.stack([ninf, ninf]))
+    assert np.all(O == 0.0) and np.all(np.isneginf(L))
+    # LSE ln 1 and ln 3 (then both shifted to ~1000): weights 1/4 and 3/4, LSE ln 4 (+shift)
+    for shift in (0.0, 1000.0):
+        la, lb = np.full(6, shift), np.full(6, shift + math.log(3.0))
+        O, L = merge(np.stack([o1, o2]), np.stack([la, lb]))
+        # (at 1000 the inputs carry ulp(1000) ~ 1e-13 of representation error)
+        assert np.max(np.abs(O - (0.25 * o1 + 0.75 * o2))) < 1e-12, shift
+        assert np.max(np.abs(L - (shift + math.log(4.0)))) < 1e-12, shift

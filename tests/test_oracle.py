@@ -61,6 +61,18 @@ def test_golden_closed_forms():
     pins.pin_golden_closed_forms(fwd, bwd)
 
 
+def test_key_slice_brute_force():
+    pins.pin_key_slice_brute_force(fwd)
+
+
+def test_merge_partition_equals_direct():
+    pins.pin_merge_partition(fwd, ora.lse_merge)
+
+
+def test_merge_closed_forms():
+    pins.pin_merge_closed_forms(ora.lse_merge)
+
+
 def test_batched_wrappers_match_heads():
     r = np.random.default_rng(12)
     q, k, v, do = r.standard_normal((4, 2, 3, 40, 8))
@@ -172,4 +184,47 @@ def test_planted_backward_mistake_is_caught(kind):
     b = _mut_bwd(kind)
     checks = [lambda: pins.pin_finite_differences(b, fwd), lambda: pins.pin_golden_closed_forms(fwd, b),
               lambda: pins.pin_torch_sdpa(fwd, b), lambda: pins.pin_single_key(fwd, b)]
+    assert any(_fails(c) for c in checks), f"no pin caught the planted mistake {kind}"
+
+
+def _mut_slice_fwd(kind):
+    """Forward over a key slice with the offset mishandled."""
+    def f(q, k, v, scale, causal=False, blockmask=None, return_p=False, tile=128, key_offset=0):
+        off = {"offset_ignored": 0, "offset_negated": -key_offset}.get(kind, key_offset)
+        return fwd(q, k, v, scale, causal, blockmask, return_p=return_p, tile=tile, key_offset=off)
+    return f
+
+
+def _mut_merge(kind):
+    def m(o_parts, lse_parts):
+        o_parts = np.asarray(o_parts, np.float64)
+        lse_parts = np.asarray(lse_parts, np.float64)
+        if kind == "no_max_shift":
+            w = np.exp(lse_parts)
+        else:
+            mx = lse_parts.max(axis=0)
+            ref = np.where(np.isfinite(mx), mx, 0.0)
+            w = np.exp(ref[None] - lse_parts) if kind == "weight_sign" else np.exp(lse_parts - ref[None])
+        tot = w.sum(axis=0)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            lse = np.log(tot) if kind == "no_max_shift" else np.where(tot > 0, np.log(tot) + ref, -np.inf)
+            frac = w if kind == "unnormalised" else w / tot[None]
+        if kind == "lse_mean":
+            lse = lse_parts.mean(axis=0)
+        O = (np.nan_to_num(frac)[..., None] * o_parts).sum(axis=0)
+        return O, lse
+    return m
+
+
+@pytest.mark.parametrize("kind", ["offset_ignored", "offset_negated"])
+def test_planted_key_offset_mistake_is_caught(kind):
+    f = _mut_slice_fwd(kind)
+    checks = [lambda: pins.pin_key_slice_brute_force(f), lambda: pins.pin_merge_partition(f, ora.lse_merge)]
+    assert any(_fails(c) for c in checks), f"no pin caught the planted mistake {kind}"
+
+
+@pytest.mark.parametrize("kind", ["no_max_shift", "weight_sign", "unnormalised", "lse_mean"])
+def test_planted_merge_mistake_is_caught(kind):
+    m = _mut_merge(kind)
+    checks = [lambda: pins.pin_merge_partition(fwd, m), lambda: pins.pin_merge_closed_forms(m)]
     assert any(_fails(c) for c in checks), f"no pin caught the planted mistake {kind}"
