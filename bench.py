@@ -2,8 +2,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One step is one pass of the whole hot path over one batch: fa_fwd (O, LSE) followed by
-fa_bwd (row preprocess, fused main backward kernel, dQ conversion).  Inputs are seeded
+One step is one pass of the whole hot path over one batch: fa_fwd (O, LSE) -- or, on the
+workloads whose heads are too few to fill the GPU, fa_fwd_splitkv (split forward + LSE
+merge) -- followed by fa_bwd (row preprocess, fused main backward kernel, dQ conversion).  Inputs are seeded
 synthetic bf16 N(0, 1) tensors of the workload's shape (no dataset exists for this
 kernel); FLOPs follow the workload convention: 4*B*H*N^2*d forward, 2.5x that backward,
 halved for causal masking.
@@ -261,6 +262,18 @@ def run_ours(args, w, world, rank, local):
     wsb = fa.fa_bwd_workspace_bytes(B, H, N, D)
     ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    splits = None
+    if w.fwd_splits is not None:
+        splits = w.fwd_splits or fa.fa_splitkv_choose(B, H, N, w.causal,
+                                                      torch.cuda.get_device_properties(dev).multi_processor_count)
+        wsfb = fa.fa_fwd_splitkv_workspace_bytes(B, H, N, D, splits)
+        wsf = torch.empty(wsfb, dtype=torch.uint8, device=dev)
+
+    def forward(q, k, v, o_, lse_):
+        if splits is None:
+            fa.fa_fwd(q, k, v, o_, lse_, B, H, N, D, scale, w.causal, mask, stream)
+        else:
+            fa.fa_fwd_splitkv(q, k, v, o_, lse_, B, H, N, D, scale, w.causal, mask, splits, wsf, wsfb, stream)
     in_bytes = sum(t.numel() * t.element_size() for t in d.values())
 
     ev_f = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -271,7 +284,7 @@ def run_ours(args, w, world, rank, local):
     def step(timed_kernels=None):
         if timed_kernels is not None:
             timed_kernels["f0"].record(stream)
-        fa.fa_fwd(d["q"], d["k"], d["v"], o, lse, B, H, N, D, scale, w.causal, mask, stream)
+        forward(d["q"], d["k"], d["v"], o, lse)
         launches[0] += fa.fa_last_launch_count()
         if timed_kernels is not None:
             timed_kernels["f1"].record(stream)
@@ -360,7 +373,7 @@ def run_ours(args, w, world, rank, local):
             stream.wait_event(ev_up[b])
             if k >= 2:
                 stream.wait_event(ev_down[b])        # step k-2's results are on the host
-            fa.fa_fwd(din["q"], din["k"], din["v"], dres["o"], dres["lse"], B, H, N, D, scale, w.causal, mask, stream)
+            forward(din["q"], din["k"], din["v"], dres["o"], dres["lse"])
             fa.fa_bwd(din["q"], din["k"], din["v"], dres["o"], dres["lse"], din["dout"], dres["dq"], dres["dk"],
                       dres["dv"], B, H, N, D, scale, w.causal, mask, ws, wsb, stream)
             ev_comp[b].record(stream)
@@ -405,6 +418,8 @@ def run_ours(args, w, world, rank, local):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(w, world),
+                       **({"fwd_splits": splits, "fwd": "fa_fwd_splitkv (split forward + LSE merge, "
+                           "both inside the fwd timing)"} if splits is not None else {}),
                        l2=f"inputs {in_bytes / 2**20:.0f} MiB per rank > 126 MiB L2, no flush"
                        if in_bytes > L2_BYTES else "inputs fit in L2"),
         "fwd_tflops": fwd_tflops, "fwd_ms": fwd_ms, "bwd_main_tflops": bmain_tflops, "bwd_main_ms": bmain_ms,
@@ -434,11 +449,17 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fwd-splits", type=int, default=None,
+                    help="forward through fa_fwd_splitkv with this many key ranges (0: chosen for the "
+                         "GPU; default: the workload's own setting)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from exact_attention_111_b200.inputs import workloads
     w = workloads()[args.workload]
+    if args.fwd_splits is not None:
+        import dataclasses
+        w = dataclasses.replace(w, fwd_splits=args.fwd_splits)
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -3,9 +3,12 @@
 The binding marshals arguments only; every step of the computation runs in the CUDA
 kernels behind the C ABI of ``include/fa.h``.  The C entry points are mirrored one to one
 (``fa_fwd``, ``fa_bwd``, ``fa_fwd_ex``, ``fa_bwd_ex``, ``fa_bwd_workspace_bytes``,
-``fa_check_status``, ``fa_status_string``, ``fa_last_launch_count``); they take torch
-tensors (or raw device addresses as ints).  ``attention_forward`` / ``attention_backward``
-and ``FlashAttention`` add output allocation with torch on top.
+``fa_bwd_noalloc``, ``fa_fwd_partial``, ``fa_lse_merge``, ``fa_fwd_splitkv``,
+``fa_fwd_splitkv_workspace_bytes``, ``fa_splitkv_choose``, ``fa_check_status``,
+``fa_status_string``, ``fa_last_launch_count``); they take torch tensors (or raw device
+addresses as ints).  ``attention_forward`` / ``attention_backward`` /
+``attention_forward_splitkv`` / ``attention_forward_partial`` / ``lse_merge`` and
+``FlashAttention`` add output allocation with torch on top.
 
 There is no fallback: if ``libfa.so`` is missing or a call fails, an exception is raised.
 """
@@ -18,12 +21,16 @@ import os
 __all__ = [
     "FAError", "fa_fwd", "fa_bwd", "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_workspace_bytes",
     "fa_check_status", "fa_status_string", "fa_last_launch_count", "fa_bwd_noalloc", "lib", "library_path",
-    "attention_forward", "attention_backward", "FlashAttention", "FA_BF16", "FA_FP16",
+    "attention_forward", "attention_backward", "FlashAttention", "FA_BF16", "FA_FP16", "FA_FP32",
+    "fa_fwd_partial", "fa_lse_merge", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes",
+    "fa_splitkv_choose", "attention_forward_splitkv", "attention_forward_partial", "lse_merge",
+    "FA_MAX_PARTS",
 ]
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
-FA_BF16, FA_FP16 = 0, 1
+FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
 TILE = 128
+FA_MAX_PARTS = 64
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libfa.so")
@@ -50,6 +57,13 @@ class BwdArgs(ctypes.Structure):
                 ("blockmask", _vp), ("dtype", _i), ("visit_log", _vp),
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("stream", _vp),
                 ("main_start_event", _vp), ("main_stop_event", _vp)]
+
+
+class PartialArgs(ctypes.Structure):
+    """Mirror of fa_fwd_partial_args."""
+    _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("o_part", _vp), ("lse_part", _vp),
+                ("B", _i), ("H", _i), ("N", _i), ("Nk", _i), ("d", _i), ("key_offset", _i),
+                ("scale", _f), ("causal", _i), ("blockmask", _vp), ("dtype", _i), ("stream", _vp)]
 
 
 class FAError(RuntimeError):
@@ -84,6 +98,16 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_noalloc.restype = _i
     L.fa_last_launch_count.argtypes = []
     L.fa_last_launch_count.restype = _i
+    L.fa_fwd_partial.argtypes = [ctypes.POINTER(PartialArgs)]
+    L.fa_fwd_partial.restype = _i
+    L.fa_lse_merge.argtypes = [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+    L.fa_lse_merge.restype = _i
+    L.fa_fwd_splitkv.argtypes = [_vp] * 5 + [_i, _i, _i, _i, _f, _i, _vp, _i, _vp, ctypes.c_size_t, _vp]
+    L.fa_fwd_splitkv.restype = _i
+    L.fa_fwd_splitkv_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+    L.fa_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
+    L.fa_splitkv_choose.argtypes = [_i, _i, _i, _i, _i]
+    L.fa_splitkv_choose.restype = _i
     _lib = L
     return L
 
@@ -155,6 +179,39 @@ def fa_fwd_ex(q, k, v, o, lse, B, H, N, d, scale, causal=False, blockmask=None, 
     _check(lib().fa_fwd_ex(ctypes.byref(a)), "fa_fwd_ex")
 
 
+def fa_fwd_partial(q, k, v, o_part, lse_part, B, H, N, Nk, d, key_offset, scale, causal=False,
+                   blockmask=None, dtype=FA_BF16, stream=None):
+    a = PartialArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, H, N, Nk, d, key_offset,
+                    scale, int(bool(causal)), _ptr(blockmask), dtype, _stream(stream))
+    _check(lib().fa_fwd_partial(ctypes.byref(a)), "fa_fwd_partial")
+
+
+def fa_lse_merge(o_parts, lse_parts, o, lse, B, H, N, d, out_dtype=FA_BF16, stream=None):
+    """o_parts / lse_parts: sequences of device tensors (or addresses), one per part."""
+    n = len(o_parts)
+    if len(lse_parts) != n:
+        raise ValueError("o_parts and lse_parts differ in length")
+    po = (_vp * max(n, 1))(*[_ptr(x) for x in o_parts])
+    pl = (_vp * max(n, 1))(*[_ptr(x) for x in lse_parts])
+    _check(lib().fa_lse_merge(po, pl, n, _ptr(o), _ptr(lse), B, H, N, d, out_dtype, _stream(stream)),
+           "fa_lse_merge")
+
+
+def fa_fwd_splitkv_workspace_bytes(B: int, H: int, N: int, d: int, num_splits: int) -> int:
+    return lib().fa_fwd_splitkv_workspace_bytes(B, H, N, d, num_splits)
+
+
+def fa_splitkv_choose(B: int, H: int, N: int, causal: bool, num_sms: int) -> int:
+    return lib().fa_splitkv_choose(B, H, N, int(bool(causal)), num_sms)
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, H, N, d, scale, causal, blockmask, num_splits, workspace,
+                   workspace_bytes, stream=None):
+    _check(lib().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
+                                int(bool(causal)), _ptr(blockmask), num_splits, _ptr(workspace),
+                                workspace_bytes, _stream(stream)), "fa_fwd_splitkv")
+
+
 def _event(e):
     if e is None or isinstance(e, int):
         return e
@@ -201,6 +258,59 @@ def attention_forward(q, k, v, causal=False, blockmask=None, scale=None, o_fp32=
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     fa_fwd_ex(q, k, v, o, lse, B, H, N, d, scale, causal, blockmask, _dtype_code(q), o_fp32,
               visit_log, stream)
+    return o, lse
+
+
+def attention_forward_splitkv(q, k, v, causal=False, blockmask=None, scale=None, num_splits=None,
+                              workspace=None, stream=None):
+    """fa_fwd_splitkv on bf16 [B, H, N, d] tensors.  ``num_splits=None`` takes
+    fa_splitkv_choose for this GPU's SM count.  Returns (O, LSE, num_splits)."""
+    import torch
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    if num_splits is None:
+        sms = torch.cuda.get_device_properties(q.device).multi_processor_count
+        num_splits = fa_splitkv_choose(B, H, N, causal, sms)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    nbytes = fa_fwd_splitkv_workspace_bytes(B, H, N, d, num_splits)
+    if workspace is None and num_splits > 1:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    fa_fwd_splitkv(q, k, v, o, lse, B, H, N, d, scale, causal, blockmask, num_splits, workspace,
+                   0 if workspace is None else workspace.numel(), stream)
+    return o, lse, num_splits
+
+
+def attention_forward_partial(q, k, v, key_offset=0, causal=False, blockmask=None, scale=None,
+                              stream=None):
+    """Attention of all query rows of q [B, H, N, d] over the keys k, v [B, H, Nk, d] that sit
+    at query-sequence positions key_offset.. (fa_fwd_partial).  Returns fp32 (O_part, LSE_part)."""
+    import torch
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    Nk = k.shape[2]
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    o = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fa_fwd_partial(q, k, v, o, lse, B, H, N, Nk, d, key_offset, scale, causal, blockmask,
+                   _dtype_code(q), stream)
+    return o, lse
+
+
+def lse_merge(o_parts, lse_parts, out_dtype=None, stream=None):
+    """Merge fp32 partial results [B, H, N, d] / [B, H, N] over disjoint key slices
+    (fa_lse_merge).  ``out_dtype``: torch dtype of O (bf16 default, fp16 or fp32)."""
+    import torch
+    B, H, N, d = o_parts[0].shape
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    code = {torch.bfloat16: FA_BF16, torch.float16: FA_FP16, torch.float32: FA_FP32}[out_dtype]
+    for t in list(o_parts) + list(lse_parts):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.float32):
+            raise ValueError("parts must be contiguous fp32 CUDA tensors")
+    o = torch.empty((B, H, N, d), dtype=out_dtype, device=o_parts[0].device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=o_parts[0].device)
+    fa_lse_merge(list(o_parts), list(lse_parts), o, lse, B, H, N, d, code, stream)
     return o, lse
 
 

@@ -24,6 +24,12 @@
 // The FA-2 idea of spreading one head over SMs ("改进并行性") is the grid over query tiles;
 // its warp repartition to cut shared-memory exchange ("优化块内工作划分") becomes the
 // per-row softmax on TMEM lanes, which needs no cross-warp reduction at all.
+//
+// Key slices.  K/V may hold Nk keys that sit at query-sequence tile kt_off onwards (one GPU's
+// shard of a sequence-sharded forward), and the key tiles may be cut into n_splits ranges of
+// split_tiles tiles, one CTA per (query pair, range), when there are too few query tiles to
+// fill the GPU.  Each range then writes its own normalised O and LSE (fp32) for a separate
+// merge kernel to combine; causal and block masks compare query-sequence positions.
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -72,8 +78,10 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = warp_id(), lane = lane_id();
   // CTAs resident together work on a few heads (their K/V tiles then come from L2), and
   // within that group the heaviest query units run first (causal: the last ones).
-  int bh, ui;
-  cta_order(blockIdx.x, a.BH, a.n_units, a.group_heads, bh, ui);
+  int bh, slot;
+  cta_order(blockIdx.x, a.BH, a.n_units * a.n_splits, a.group_heads, bh, slot);
+  int ui = slot / a.n_splits;
+  const int split = slot - ui * a.n_splits;     // key-tile range of this CTA
   if (a.causal) ui = a.n_units - 1 - ui;
   const int qt0 = 2 * ui;
   const DevStatus st{a.status, a.timeout_ns};
@@ -99,16 +107,19 @@ __global__ void __launch_bounds__(320, 1)
     tmem_relinquish();
   }
   if (warp == 8) {
-    // Union list of key tiles needed by either query tile, with per-tile keep bits.
+    // Union list of this range's key tiles needed by either query tile, with per-tile keep
+    // bits; entries hold the K/V tile index, the masks see its query-sequence tile jg.
     int count = 0, c0 = 0, c1 = 0;
-    for (int base = 0; base < a.T; base += 32) {
+    const int jb = split * a.split_tiles;
+    const int je = min(a.Tk, jb + a.split_tiles);
+    for (int base = jb; base < je; base += 32) {
       const int j = base + lane;
       bool k0 = false, k1 = false;
-      if (j < a.T) {
-        const int qa = qt0, qb = qt0 + 1;
-        k0 = (!a.causal || j <= qa) && (a.blockmask == nullptr || a.blockmask[(size_t)qa * a.T + j] != 0);
-        k1 = qb < a.T && (!a.causal || j <= qb) &&
-             (a.blockmask == nullptr || a.blockmask[(size_t)qb * a.T + j] != 0);
+      if (j < je) {
+        const int qa = qt0, qb = qt0 + 1, jg = a.kt_off + j;
+        k0 = (!a.causal || jg <= qa) && (a.blockmask == nullptr || a.blockmask[(size_t)qa * a.T + jg] != 0);
+        k1 = qb < a.T && (!a.causal || jg <= qb) &&
+             (a.blockmask == nullptr || a.blockmask[(size_t)qb * a.T + jg] != 0);
       }
       const unsigned bal = __ballot_sync(0xffffffffu, k0 || k1);
       if (k0 || k1) list[count + __popc(bal & ((1u << lane) - 1u))] = j | (int(k0) << 16) | (int(k1) << 17);
@@ -207,7 +218,7 @@ __global__ void __launch_bounds__(320, 1)
             }
             tc_commit(&sh.s_full[q]);
             if (a.visit != nullptr)
-              atomicAdd(&a.visit[((size_t)bh * a.T + (qt0 + q)) * a.T + (ec & 0xFFFF)], 1);
+              atomicAdd(&a.visit[((size_t)bh * a.T + (qt0 + q)) * a.T + a.kt_off + (ec & 0xFFFF)], 1);
           }
           return true;
         };
@@ -240,7 +251,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int u = 0; u < nu; ++u) {
       const int e = list[u];
       if (!((e >> (16 + q)) & 1)) continue;
-      const int key0 = (e & 0xFFFF) * kTile;
+      const int key0 = (e & 0xFFFF) * kTile;          // first K/V row of the tile
+      const int kpos0 = key0 + a.kt_off * kTile;      // its query-sequence position
       ok = mbar_wait(&sh.s_full[q], c & 1, abort_flag, st);
       if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
       tc_fence_after();
@@ -255,9 +267,9 @@ __global__ void __launch_bounds__(320, 1)
       float s[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
-      if ((a.causal && key0 + kTile - 1 > qt * kTile) || key0 + kTile > a.N) {
-        int lim = a.N - key0;                         // keys at or beyond N do not exist
-        if (a.causal) lim = min(lim, row - key0 + 1); // key <= row
+      if ((a.causal && kpos0 + kTile - 1 > qt * kTile) || key0 + kTile > a.Nk) {
+        int lim = a.Nk - key0;                         // K/V rows at or beyond Nk do not exist
+        if (a.causal) lim = min(lim, row - kpos0 + 1); // key position <= row
 #pragma unroll
         for (int i = 0; i < 128; ++i)
           if (i >= lim) s[i] = -INFINITY;
@@ -331,8 +343,9 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const bool valid = row < a.N;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      if (valid) a.lse[(size_t)bh * a.N + row] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
-      const size_t obase = ((size_t)bh * a.N + row) * D;
+      if (valid)
+        a.lse[split * a.lse_split_stride + (size_t)bh * a.N + row] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+      const size_t obase = split * a.o_split_stride + ((size_t)bh * a.N + row) * D;
 #pragma unroll
       for (int cc = 0; cc < D; cc += 32) {
         uint32_t o[32];
@@ -378,11 +391,11 @@ template <int D, bool kFp16>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdArgs& a,
                          cudaStream_t s) {
   using C = FwdCfg<D>;
-  const size_t smem = C::kSmemTiles + (size_t)a.T * sizeof(int) + 1024;
+  const size_t smem = C::kSmemTiles + (size_t)min(a.Tk, a.split_tiles) * sizeof(int) + 1024;
   auto kern = fwd_kernel<D, kFp16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.n_units);
+  const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.n_units) * static_cast<unsigned>(a.n_splits);
   kern<<<grid, C::kThreads, smem, s>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }

@@ -83,6 +83,44 @@ int check_shape(int B, int H, int N, int d, float scale, int dtype) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// The forward's grid is BH x units x splits CTAs, indexed by an int.
+bool fwd_grid_ok(int BH, int units, int splits) {
+  return (long long)BH * units * splits <= (long long)0x7fffffff;
+}
+
+// Self-attention forward arguments over all T key tiles as one range.
+void self_fwd_args(FwdArgs& a, int BH, int N) {
+  const int T = (N + kTile - 1) / kTile;
+  a.N = N;
+  a.BH = BH;
+  a.T = T;
+  a.n_units = (T + 1) / 2;
+  a.Nk = N;
+  a.Tk = T;
+  a.kt_off = 0;
+  a.n_splits = 1;
+  a.split_tiles = T;
+  a.o_split_stride = 0;
+  a.lse_split_stride = 0;
+  a.group_heads = group_heads_for(BH, a.n_units);
+}
+
+struct SplitLayout {
+  size_t o_parts, lse_parts, total;
+  long long o_stride, lse_stride;   // elements between consecutive parts
+};
+
+SplitLayout split_layout(int B, int H, int N, int d, int S) {
+  const size_t rows = (size_t)B * H * N;
+  SplitLayout w;
+  w.o_parts = 0;
+  w.o_stride = (long long)(align256(rows * d * 4) / 4);
+  w.lse_parts = align256(rows * d * 4) * S;
+  w.lse_stride = (long long)(align256(rows * 4) / 4);
+  w.total = w.lse_parts + align256(rows * 4) * S;
+  return w;
+}
+
 struct WsLayout {
   size_t dq_acc, delta, lse2, total;
 };
@@ -155,6 +193,7 @@ int fa_fwd_ex(const fa_fwd_args* p) {
   const bool fp16 = x.dtype == FA_FP16;
   const int BH = x.B * x.H;
   const int T = (x.N + kTile - 1) / kTile;
+  if (!fwd_grid_ok(BH, (T + 1) / 2, 1)) return FA_ERR_UNSUPPORTED;
   if (!get_encode()) return FA_ERR_CUDA;
   CUtensorMap tq, tk, tv;
   if (!encode_qkv(&tq, x.q, BH, x.N, x.d, fp16) || !encode_qkv(&tk, x.k, BH, x.N, x.d, fp16) ||
@@ -167,11 +206,7 @@ int fa_fwd_ex(const fa_fwd_args* p) {
   a.visit = x.visit_log;
   if (status_word(&a.status) != FA_OK) return FA_ERR_CUDA;
   a.timeout_ns = kWaitLimitNs;
-  a.N = x.N;
-  a.BH = BH;
-  a.T = T;
-  a.n_units = (T + 1) / 2;
-  a.group_heads = group_heads_for(BH, a.n_units);
+  self_fwd_args(a, BH, x.N);
   a.causal = x.causal != 0;
   a.o_fp32 = x.o_fp32 != 0;
   a.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
@@ -259,6 +294,162 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   a.dtype = FA_BF16; a.visit_log = nullptr;
   a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.stream = stream;
   return fa_bwd_ex(&a);
+}
+
+int fa_fwd_partial(const fa_fwd_partial_args* p) {
+  if (p == nullptr) return FA_ERR_INVALID_ARG;
+  const fa_fwd_partial_args& x = *p;
+  int rc = check_shape(x.B, x.H, x.N, x.d, x.scale, x.dtype);
+  if (rc != FA_OK) return rc;
+  if (x.Nk < 1 || x.key_offset < 0 || x.key_offset % kTile != 0) return FA_ERR_INVALID_ARG;
+  if (x.Nk > FA_MAX_SEQLEN || (long long)x.B * x.H * x.Nk * x.d > (1LL << 46)) return FA_ERR_UNSUPPORTED;
+  if ((x.causal || x.blockmask) && (long long)x.key_offset + x.Nk > x.N) return FA_ERR_INVALID_ARG;
+  if (!x.q || !x.k || !x.v || !x.o_part || !x.lse_part) return FA_ERR_INVALID_ARG;
+  if (!aligned(x.q, 16) || !aligned(x.k, 16) || !aligned(x.v, 16) || !aligned(x.o_part, 16) ||
+      !aligned(x.lse_part, 4))
+    return FA_ERR_INVALID_ARG;
+  const bool fp16 = x.dtype == FA_FP16;
+  const int BH = x.B * x.H;
+  const int T = (x.N + kTile - 1) / kTile;
+  if (!fwd_grid_ok(BH, (T + 1) / 2, 1)) return FA_ERR_UNSUPPORTED;
+  if (!get_encode()) return FA_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (!encode_qkv(&tq, x.q, BH, x.N, x.d, fp16) || !encode_qkv(&tk, x.k, BH, x.Nk, x.d, fp16) ||
+      !encode_qkv(&tv, x.v, BH, x.Nk, x.d, fp16))
+    return FA_ERR_CUDA;
+  FwdArgs a{};
+  a.o = x.o_part;
+  a.lse = x.lse_part;
+  a.blockmask = x.blockmask;
+  a.visit = nullptr;
+  if (status_word(&a.status) != FA_OK) return FA_ERR_CUDA;
+  a.timeout_ns = kWaitLimitNs;
+  self_fwd_args(a, BH, x.N);
+  a.Nk = x.Nk;
+  a.Tk = (x.Nk + kTile - 1) / kTile;
+  a.kt_off = x.key_offset / kTile;
+  a.split_tiles = a.Tk;
+  a.causal = x.causal != 0;
+  a.o_fp32 = 1;
+  a.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
+  t_last_launches = 0;
+  if (launch_fwd(tq, tk, tv, a, x.d, fp16, static_cast<cudaStream_t>(x.stream)) != cudaSuccess) return FA_ERR_CUDA;
+  t_last_launches = 1;
+  return FA_OK;
+}
+
+int fa_lse_merge(const float* const* o_parts, const float* const* lse_parts, int n_parts, void* o, float* lse,
+                 int B, int H, int N, int d, int out_dtype, void* stream) {
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (out_dtype != FA_BF16 && out_dtype != FA_FP16 && out_dtype != FA_FP32) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * H * N * d > (1LL << 46)) return FA_ERR_UNSUPPORTED;
+  if (n_parts < 1 || n_parts > FA_MAX_PARTS) return FA_ERR_INVALID_ARG;
+  if (!o_parts || !lse_parts || !o || !lse || !aligned(o, 16) || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  MergeArgs m{};
+  for (int i = 0; i < n_parts; ++i) {
+    if (!o_parts[i] || !lse_parts[i] || !aligned(o_parts[i], 16) || !aligned(lse_parts[i], 4))
+      return FA_ERR_INVALID_ARG;
+    m.o_parts[i] = o_parts[i];
+    m.lse_parts[i] = lse_parts[i];
+  }
+  m.o = o;
+  m.lse = lse;
+  m.rows = (long long)B * H * N;
+  m.n_parts = n_parts;
+  m.out_kind = out_dtype;
+  t_last_launches = 0;
+  if (launch_merge(m, d, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  t_last_launches = 1;
+  return FA_OK;
+}
+
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int num_splits) {
+  if (check_shape(B, H, N, d, 1.f, FA_BF16) != FA_OK) return 0;
+  if (num_splits < 1 || num_splits > FA_MAX_PARTS) return 0;
+  return split_layout(B, H, N, d, num_splits).total;
+}
+
+int fa_splitkv_choose(int B, int H, int N, int causal, int num_sms) {
+  if (B < 1 || H < 1 || N < 1 || N > FA_MAX_SEQLEN || num_sms < 1) return 0;
+  const int T = (N + kTile - 1) / kTile;
+  const long long units = (long long)B * H * ((T + 1) / 2);
+  int best = 1;
+  long long best_cost = -1;
+  for (int S = 1; S <= FA_MAX_PARTS; ++S) {
+    const int sp = (T + S - 1) / S;                 // key tiles per range
+    if (S > 1 && sp < 4) break;
+    const int s_eff = (T + sp - 1) / sp;            // ranges that hold any tile
+    if (s_eff < S) continue;                        // same cut as a smaller S
+    // causal CTAs average half the tiles: the light ones free their SMs early
+    const long long load = units * s_eff / (causal ? 2 : 1);
+    const long long waves = (load + num_sms - 1) / num_sms;
+    const long long cost = (waves < 1 ? 1 : waves) * (sp + 2);
+    if (best_cost < 0 || 10 * cost < 9 * best_cost) {   // a new cut must win by 10 % (merge cost)
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                   float scale, int causal, const uint8_t* blockmask, int num_splits, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d, scale, FA_BF16);
+  if (rc != FA_OK) return rc;
+  if (num_splits < 1 || num_splits > FA_MAX_PARTS) return FA_ERR_INVALID_ARG;
+  if (num_splits == 1) return fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, blockmask, stream);
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_INVALID_ARG;
+  const SplitLayout w = split_layout(B, H, N, d, num_splits);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total) return FA_ERR_WORKSPACE;
+  const int BH = B * H;
+  const int T = (N + kTile - 1) / kTile;
+  const int sp = (T + num_splits - 1) / num_splits;
+  const int s_eff = (T + sp - 1) / sp;              // ranges past the last tile are dropped
+  if (!fwd_grid_ok(BH, (T + 1) / 2, s_eff)) return FA_ERR_UNSUPPORTED;
+  if (!get_encode()) return FA_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (!encode_qkv(&tq, q, BH, N, d, false) || !encode_qkv(&tk, k, BH, N, d, false) ||
+      !encode_qkv(&tv, v, BH, N, d, false))
+    return FA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* o_parts = reinterpret_cast<float*>(ws + w.o_parts);
+  float* lse_parts = reinterpret_cast<float*>(ws + w.lse_parts);
+  FwdArgs a{};
+  a.o = o_parts;
+  a.lse = lse_parts;
+  a.blockmask = blockmask;
+  a.visit = nullptr;
+  if (status_word(&a.status) != FA_OK) return FA_ERR_CUDA;
+  a.timeout_ns = kWaitLimitNs;
+  self_fwd_args(a, BH, N);
+  a.n_splits = s_eff;
+  a.split_tiles = sp;
+  a.o_split_stride = w.o_stride;
+  a.lse_split_stride = w.lse_stride;
+  a.group_heads = group_heads_for(BH, a.n_units * s_eff);
+  a.causal = causal != 0;
+  a.o_fp32 = 1;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  t_last_launches = 0;
+  if (launch_fwd(tq, tk, tv, a, d, false, s) != cudaSuccess) return FA_ERR_CUDA;
+  MergeArgs m{};
+  for (int i = 0; i < s_eff; ++i) {
+    m.o_parts[i] = o_parts + i * w.o_stride;
+    m.lse_parts[i] = lse_parts + i * w.lse_stride;
+  }
+  m.o = o;
+  m.lse = lse;
+  m.rows = (long long)BH * N;
+  m.n_parts = s_eff;
+  m.out_kind = FA_BF16;
+  if (launch_merge(m, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  t_last_launches = 2;
+  return FA_OK;
 }
 
 int fa_check_status(void* stream) {

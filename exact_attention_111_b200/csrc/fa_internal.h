@@ -14,17 +14,32 @@ constexpr int kMaxTiles = 2048;     // tile lists live in shared memory (N <= 20
 // Error codes a kernel can record in the device status word (read by fa_check_status).
 enum : int { kDevOk = 0, kDevTimeout = 4, kDevBadState = 6 };
 
+constexpr int kMaxParts = 64;       // most key splits / merged parts per call
+
 struct FwdArgs {
-  void* o;                  // [BH, N, d] 16-bit, or fp32 when o_fp32
-  float* lse;               // [BH, N]
+  void* o;                  // [BH, N, d] 16-bit, or fp32 when o_fp32 (split s at o + s * o_split_stride)
+  float* lse;               // [BH, N]                                (split s at lse + s * lse_split_stride)
   const uint8_t* blockmask; // [T, T] or null
   int* visit;               // [BH, T, T] or null
   int* status;              // device status word
   unsigned long long timeout_ns;
-  int N, BH, T, n_units;    // n_units = ceil(T / 2): one CTA covers two 128-row query tiles
+  int N, BH, T, n_units;    // queries; n_units = ceil(T / 2): one CTA covers two 128-row query tiles
+  int Nk, Tk;               // keys in K/V and their 128-row tiles (N and T for self-attention)
+  int kt_off;               // query-sequence tile index of key tile 0 (causal and mask use it)
+  int n_splits, split_tiles;// split s takes key tiles [s * split_tiles, (s + 1) * split_tiles)
+  long long o_split_stride, lse_split_stride;  // elements between consecutive splits' outputs
   int group_heads;          // CTAs are ordered in groups of this many heads (see cta_order)
   int causal, o_fp32;
   float scale_log2;         // scale * log2(e)
+};
+
+struct MergeArgs {
+  const float* o_parts[kMaxParts];    // each [rows, d] fp32
+  const float* lse_parts[kMaxParts];  // each [rows] fp32
+  void* o;                            // [rows, d]: bf16, fp16 or fp32 (out_kind 0, 1, 2)
+  float* lse;                         // [rows]
+  long long rows;
+  int n_parts, out_kind;
 };
 
 struct BwdPreArgs {
@@ -69,6 +84,7 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int d, bool fp16,
                        cudaStream_t s);
 cudaError_t launch_bwd_post(const BwdPostArgs& a, bool fp16, cudaStream_t s);
+cudaError_t launch_merge(const MergeArgs& a, int d, cudaStream_t s);
 
 int* device_status_word();  // address of the per-process device status word
 

@@ -35,6 +35,7 @@ class Workload:
     k_scale: float = 1.0
     butterfly: bool = False
     seed: int = 0
+    fwd_splits: int | None = None   # None: plain forward; 0: split-KV, count chosen; n: n ranges
     extra: dict = field(default_factory=dict, compare=False)
 
     @property
@@ -47,7 +48,10 @@ class Workload:
 
 
 def workloads() -> dict[str, Workload]:
-    """The five workload families, named by what they are and their sizes."""
+    """The workload families, named by what they are and their sizes: the single head, the
+    GPT-2-shaped batch, the sequence-length sweep, the long peaked-causal context, the
+    butterfly block-sparse batch, and one long head too few query tiles to fill the GPU
+    (the split-KV forward's case)."""
     w: dict[str, Workload] = {}
     w["head_N128_d64"] = Workload("head_N128_d64", 1, 1, 128, 64, seed=1001)
     w["gpt2_B64_H16_N1024_d64"] = Workload("gpt2_B64_H16_N1024_d64", 64, 16, 1024, 64, seed=1002)
@@ -61,6 +65,9 @@ def workloads() -> dict[str, Workload]:
         "long_B1_H32_N16384_d128_causal_k4", 1, 32, 16384, 128, causal=True, k_scale=4.0, seed=1004)
     w["butterfly_B8_H16_N4096_d64"] = Workload(
         "butterfly_B8_H16_N4096_d64", 8, 16, 4096, 64, butterfly=True, seed=1005)
+    for causal in (False, True):
+        name = f"splitkv_B1_H1_N16384_d128{'_causal' if causal else ''}"
+        w[name] = Workload(name, 1, 1, 16384, 128, causal=causal, seed=1006, fwd_splits=0)
     return w
 
 

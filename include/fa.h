@@ -44,7 +44,11 @@ typedef enum {
   FA_ERR_WORKSPACE = 5      /* workspace pointer NULL/misaligned or smaller than required   */
 } fa_status;
 
-typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+typedef enum {
+  FA_BF16 = 0,
+  FA_FP16 = 1,
+  FA_FP32 = 2              /* output type of fa_lse_merge only */
+} fa_dtype;
 
 /* Largest sequence length accepted (tile lists live in shared memory: T <= 2048). */
 #define FA_MAX_SEQLEN (2048 * 128)
@@ -154,6 +158,94 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    const void* dout, void* dq, void* dk, void* dv,
                    int B, int H, int N, int d, float scale, int causal, const uint8_t* blockmask,
                    void* stream);
+
+/*
+ * ---------------------------------------------------------------------------------------
+ * Attention over a slice of the keys, and the merge of slices (split-KV forward).
+ *
+ * The FlashAttention-2 wiki ("改进并行性") spreads one head's work over the GPU's SMs because
+ * long sequences with small batches otherwise leave SMs idle; the NeurIPS22 summary leaves
+ * decode-style small-batch long-context use and multi-GPU sequence parallelism to follow-on
+ * work ("边界条件", "局限与 Future Work").  Cutting the KEYS of a head into slices serves both:
+ * each slice's attention is independent, and the results combine exactly through their
+ * log-sum-exps (the online-softmax rescaling of "核心方法 / Tiling 与 online softmax"):
+ *     LSE = ln sum_s exp(LSE_s),    O = sum_s exp(LSE_s - LSE) O_s.
+ * ---------------------------------------------------------------------------------------
+ */
+
+/* Most key splits of fa_fwd_splitkv and most parts of fa_lse_merge. */
+#define FA_MAX_PARTS 64
+
+/*
+ * Forward over a slice of the keys: every query row of q attends only to the Nk keys of k/v.
+ *   q          : in,  [B, H, N, d] (dtype), all query rows of the sequence
+ *   k, v       : in,  [B, H, Nk, d] (dtype), key rows that sit at query-sequence positions
+ *                key_offset .. key_offset + Nk - 1
+ *   o_part     : out, [B, H, N, d] fp32, normalised over this slice's keys (0 where a row
+ *                sees none of them)
+ *   lse_part   : out, [B, H, N] fp32, natural log-sum-exp over this slice (-inf if none)
+ *   key_offset : a multiple of 128, >= 0.  causal keeps key position <= query row; the
+ *                blockmask ([T, T], T = ceil(N / 128), as for fa_fwd) is indexed by the
+ *                query-sequence tiles of the keys.  With causal or a blockmask,
+ *                key_offset + Nk must not exceed N; without either, Nk and key_offset are
+ *                free (cross-attention over any key set).
+ * One launch.  Errors: FA_ERR_INVALID_ARG for NULL or misaligned pointers, Nk < 1, a bad
+ * key_offset; otherwise as fa_fwd.
+ */
+typedef struct {
+  const void* q; const void* k; const void* v;
+  float* o_part;
+  float* lse_part;
+  int B, H, N, Nk, d;
+  int key_offset;
+  float scale;
+  int causal;
+  const uint8_t* blockmask;
+  int dtype;               /* fa_dtype of q, k, v: FA_BF16 or FA_FP16 */
+  void* stream;
+} fa_fwd_partial_args;
+
+int fa_fwd_partial(const fa_fwd_partial_args* args);
+
+/*
+ * Combine n_parts results over disjoint key slices of the same rows.
+ *   o_parts, lse_parts : HOST arrays of n_parts DEVICE pointers; part s is fp32
+ *                        [B, H, N, d] and fp32 [B, H, N], 16- and 4-byte aligned.  The
+ *                        pointers may address another GPU's memory where peer access is
+ *                        enabled (the kernel reads them with plain loads).
+ *   o                  : out, [B, H, N, d] of out_dtype (FA_BF16, FA_FP16 or FA_FP32)
+ *   lse                : out, [B, H, N] fp32
+ * 1 <= n_parts <= FA_MAX_PARTS.  A row no part saw a key for gets O = 0 and LSE = -inf.
+ * One launch; nothing is allocated.
+ */
+int fa_lse_merge(const float* const* o_parts, const float* const* lse_parts, int n_parts,
+                 void* o, float* lse, int B, int H, int N, int d, int out_dtype, void* stream);
+
+/*
+ * Split-KV forward: the same result as fa_fwd (bf16), computed with the key tiles of every
+ * head cut into num_splits ranges of ceil(T / num_splits) tiles, one CTA per (pair of query
+ * tiles, range), and merged.  For heads too few to fill the GPU (small batch, long N).
+ *   num_splits : 1 .. FA_MAX_PARTS (1 = fa_fwd itself: one launch, no workspace used);
+ *                fa_splitkv_choose gives a good value
+ *   workspace  : device scratch of fa_fwd_splitkv_workspace_bytes(B, H, N, d, num_splits)
+ *                bytes, 256-byte aligned (the fp32 partial O and LSE of every range)
+ * Two launches (the split forward, then the merge) when num_splits > 1.  LSE and O equal
+ * fa_fwd's up to fp32 rounding of the merge; ranges past the last key tile are empty and
+ * cost one short CTA each.
+ */
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int num_splits);
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int H, int N, int d, float scale, int causal, const uint8_t* blockmask,
+                   int num_splits, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Host arithmetic: the split count fa_fwd_splitkv should use on a GPU with num_sms SMs (one
+ * forward CTA per SM).  Minimises (waves of CTAs) x (key tiles per CTA + 2), the 2 standing
+ * for a CTA's fixed cost in tiles and causal CTAs counting half, over 1 .. FA_MAX_PARTS
+ * with at least 4 key tiles per range; a larger count must win by 10 % (the merge's cost).  Returns 1 when the query tiles alone fill the GPU, and 0
+ * for invalid sizes.
+ */
+int fa_splitkv_choose(int B, int H, int N, int causal, int num_sms);
 
 /* Static human-readable name of a status code. */
 const char* fa_status_string(int status);

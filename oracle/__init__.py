@@ -6,6 +6,7 @@ from .attention import (  # noqa: F401
     attention_fwd,
     attention_fwd_head,
     attention_fwd_partial,
+    attention_fwd_rows,
     attention_fwd_head_tiled,
     lse_merge,
     softmax_rows,

@@ -232,3 +232,19 @@ def attention_fwd_partial(q, k, v, scale: float, causal: bool = False, blockmask
         O[b, h], L[b, h] = attention_fwd_head(q[b, h], k[b, h], v[b, h], scale, causal, bm,
                                               key_offset=key_offset)
     return O, L
+
+
+def attention_fwd_rows(q, k, v, scale: float, causal: bool, rows):
+    """One head, only the query rows ``rows`` (no block mask): (O [len(rows), d], LSE).
+    A row's output depends only on its own query and the keys it sees, so evaluating a
+    sample of rows is exact -- used to check full-size problems whose N x N matrices do not
+    fit in memory."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    rows = np.asarray(rows)
+    S = scale * (q[rows] @ k.T)
+    if causal:
+        S = np.where(np.arange(k.shape[0])[None, :] <= rows[:, None], S, -np.inf)
+    P, _, _, lse = softmax_rows(S)
+    return P @ v, lse

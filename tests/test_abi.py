@@ -122,3 +122,107 @@ def test_python_binding_raises(L):
     with pytest.raises(fa.FAError) as e:
         fa.fa_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 96, 0.125, False, None, stream=0)
     assert e.value.code == fa.FA_ERR_UNSUPPORTED
+
+
+# ----------------------------------------------------------------------------------------
+# Split-KV forward, forward over a key slice, LSE merge
+# ----------------------------------------------------------------------------------------
+
+def test_splitkv_symbols_declared():
+    names = declared_functions()
+    for n in ("fa_fwd_partial", "fa_lse_merge", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes",
+              "fa_splitkv_choose"):
+        assert n in names, n
+
+
+def test_splitkv_workspace_formula(L):
+    a = lambda x: (x + 255) // 256 * 256
+    for B, H, N, d, S in ((1, 1, 16384, 128, 2), (2, 3, 1000, 64, 5), (1, 1, 1, 64, 1), (4, 2, 777, 128, 64)):
+        rows = B * H * N
+        assert fa.fa_fwd_splitkv_workspace_bytes(B, H, N, d, S) == S * (a(rows * d * 4) + a(rows * 4))
+    assert fa.fa_fwd_splitkv_workspace_bytes(1, 1, 128, 64, 0) == 0
+    assert fa.fa_fwd_splitkv_workspace_bytes(1, 1, 128, 64, 65) == 0
+    assert fa.fa_fwd_splitkv_workspace_bytes(1, 1, 128, 96, 2) == 0
+
+
+def _choose_model(B, H, N, causal, sms):
+    """The documented rule, restated: minimise waves x (tiles per range + 2), causal CTAs
+    counting half, ranges of >= 4 tiles, a larger count winning only by 10 %."""
+    T = -(-N // 128)
+    units = B * H * -(-T // 2)
+    best, best_cost = 1, None
+    for S in range(1, 65):
+        sp = -(-T // S)
+        if S > 1 and sp < 4:
+            break
+        s_eff = -(-T // sp)
+        if s_eff < S:
+            continue
+        load = units * s_eff // (2 if causal else 1)
+        cost = max(1, -(-load // sms)) * (sp + 2)
+        if best_cost is None or 10 * cost < 9 * best_cost:
+            best, best_cost = S, cost
+    return best
+
+
+def test_splitkv_choose(L):
+    # one head of 16k keys leaves most SMs idle: two ranges; a full GPU takes none
+    assert fa.fa_splitkv_choose(1, 1, 16384, False, 148) == 2
+    assert fa.fa_splitkv_choose(64, 16, 1024, False, 148) == 1
+    assert fa.fa_splitkv_choose(4, 32, 4096, True, 148) == 1
+    for B, H, N, causal in ((1, 1, 4096, False), (1, 1, 16384, True), (2, 1, 8192, False),
+                            (1, 3, 30000, True), (1, 2, 16384, False), (3, 5, 300, False)):
+        for sms in (148, 132, 20):
+            got = fa.fa_splitkv_choose(B, H, N, causal, sms)
+            assert got == _choose_model(B, H, N, causal, sms), (B, H, N, causal, sms)
+            T = -(-N // 128)
+            assert 1 <= got <= 64 and (got == 1 or -(-T // got) >= 4)
+    assert fa.fa_splitkv_choose(0, 1, 128, False, 148) == 0
+    assert fa.fa_splitkv_choose(1, 1, 128, False, 0) == 0
+
+
+def test_splitkv_argument_errors(L):
+    ws = fa.fa_fwd_splitkv_workspace_bytes(1, 1, 1024, 64, 4)
+
+    def call(S=4, wsp=0x100000, wsb=ws, d=64, ptr=FAKE):
+        return L.fa_fwd_splitkv(ptr, ptr, ptr, ptr, ptr, 1, 1, 1024, d, 0.125, 0, None, S, wsp, wsb, None)
+    assert call(S=0) == fa.FA_ERR_INVALID_ARG
+    assert call(S=65) == fa.FA_ERR_INVALID_ARG
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(ptr=None) == fa.FA_ERR_INVALID_ARG
+    assert call(wsb=ws - 1) == fa.FA_ERR_WORKSPACE
+    assert call(wsp=None) == fa.FA_ERR_WORKSPACE
+    assert call(wsp=0x100000 + 64) == fa.FA_ERR_WORKSPACE
+
+
+def test_partial_argument_errors(L):
+    def call(**kw):
+        a = dict(N=1024, Nk=256, key_offset=256, causal=0, mask=None, d=64, dtype=fa.FA_BF16, k=FAKE)
+        a.update(kw)
+        args = fa.PartialArgs(FAKE, a["k"], FAKE, FAKE, FAKE, 1, 1, a["N"], a["Nk"], a["d"], a["key_offset"],
+                              0.125, a["causal"], a["mask"], a["dtype"], None)
+        return L.fa_fwd_partial(ctypes.byref(args))
+    assert call(key_offset=100) == fa.FA_ERR_INVALID_ARG        # not a multiple of 128
+    assert call(key_offset=-128) == fa.FA_ERR_INVALID_ARG
+    assert call(Nk=0) == fa.FA_ERR_INVALID_ARG
+    assert call(causal=1, key_offset=896) == fa.FA_ERR_INVALID_ARG   # keys past the sequence
+    assert call(mask=FAKE, key_offset=896) == fa.FA_ERR_INVALID_ARG
+    assert call(d=80) == fa.FA_ERR_UNSUPPORTED
+    assert call(dtype=2) == fa.FA_ERR_UNSUPPORTED                # fp32 inputs are not accepted
+    assert call(k=FAKE + 4) == fa.FA_ERR_INVALID_ARG
+    assert call(Nk=2048 * 128 + 1) == fa.FA_ERR_UNSUPPORTED
+    assert L.fa_fwd_partial(None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_merge_argument_errors(L):
+    def call(n=2, d=64, out=fa.FA_BF16, parts=None, o=FAKE):
+        ps = parts if parts is not None else [FAKE] * max(n, 1)
+        arr = (ctypes.c_void_p * len(ps))(*ps)
+        return L.fa_lse_merge(arr, arr, n, o, FAKE, 1, 1, 128, d, out, None)
+    assert call(n=0) == fa.FA_ERR_INVALID_ARG
+    assert call(n=65, parts=[FAKE] * 65) == fa.FA_ERR_INVALID_ARG
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(out=3) == fa.FA_ERR_UNSUPPORTED
+    assert call(parts=[FAKE, None]) == fa.FA_ERR_INVALID_ARG
+    assert call(parts=[FAKE, FAKE + 4]) == fa.FA_ERR_INVALID_ARG   # O part not 16-byte aligned
+    assert call(o=None) == fa.FA_ERR_INVALID_ARG

@@ -73,6 +73,16 @@ def test_merge_closed_forms():
     pins.pin_merge_closed_forms(ora.lse_merge)
 
 
+def test_row_sample_matches_whole_head():
+    r = np.random.default_rng(21)
+    q, k, v = r.standard_normal((3, 50, 6))
+    rows = np.array([0, 3, 17, 49])
+    for causal in (False, True):
+        O, L = fwd(q, k, v, 0.4, causal)
+        Os, Ls = ora.attention_fwd_rows(q, k, v, 0.4, causal, rows)
+        assert np.max(np.abs(Os - O[rows])) < 1e-13 and np.max(np.abs(Ls - L[rows])) < 1e-13
+
+
 def test_batched_wrappers_match_heads():
     r = np.random.default_rng(12)
     q, k, v, do = r.standard_normal((4, 2, 3, 40, 8))
