@@ -259,7 +259,8 @@ def run_ours(args, w, world, rank, local):
     o = torch.empty_like(d["q"])
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
-    wsb = fa.fa_bwd_workspace_bytes(B, H, N, D)
+    det = bool(args.deterministic)
+    wsb = fa.fa_bwd_workspace_bytes_ex(B, H, N, D, det)
     ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     splits = None
@@ -290,7 +291,8 @@ def run_ours(args, w, world, rank, local):
             timed_kernels["f1"].record(stream)
         fa.fa_bwd_ex(d["q"], d["k"], d["v"], o, lse, d["dout"], dq, dk, dv, B, H, N, D, scale, w.causal, mask,
                      fa.FA_BF16, None, ws, wsb, stream,
-                     timed_kernels["b0"] if timed_kernels else None, timed_kernels["b1"] if timed_kernels else None)
+                     timed_kernels["b0"] if timed_kernels else None, timed_kernels["b1"] if timed_kernels else None,
+                     deterministic=det)
         launches[0] += fa.fa_last_launch_count()
 
     # ---------------------------------------------------------------- warm-up
@@ -374,8 +376,9 @@ def run_ours(args, w, world, rank, local):
             if k >= 2:
                 stream.wait_event(ev_down[b])        # step k-2's results are on the host
             forward(din["q"], din["k"], din["v"], dres["o"], dres["lse"])
-            fa.fa_bwd(din["q"], din["k"], din["v"], dres["o"], dres["lse"], din["dout"], dres["dq"], dres["dk"],
-                      dres["dv"], B, H, N, D, scale, w.causal, mask, ws, wsb, stream)
+            fa.fa_bwd_ex(din["q"], din["k"], din["v"], dres["o"], dres["lse"], din["dout"], dres["dq"], dres["dk"],
+                         dres["dv"], B, H, N, D, scale, w.causal, mask, fa.FA_BF16, None, ws, wsb, stream,
+                         deterministic=det)
             ev_comp[b].record(stream)
             s_down.wait_event(ev_comp[b])
             with torch.cuda.stream(s_down):
@@ -407,7 +410,7 @@ def run_ours(args, w, world, rank, local):
         dom, dom_tf, dom_flops = "bwd_main", bmain_tflops, bwd_flops
     else:
         dom, dom_tf, dom_flops = "fwd", fwd_tflops, fwd_flops
-    traffic = stored_traffic(dom, w.name)
+    traffic = stored_traffic(dom, w.name) if not det else None   # captured for the default mode only
     roofline = {"bound": "tensor", "achieved": dom_tf, "peak": peak_sust, "unit": "TFLOP/s",
                 "frac": dom_tf / peak_sust, "traffic": traffic, "kernel": dom,
                 "peak_source": f"bf16_tflops_sustained of {peak_src} (MEASURED_PEAKS.json)",
@@ -420,6 +423,7 @@ def run_ours(args, w, world, rank, local):
         "config": dict(workload_config(w, world),
                        **({"fwd_splits": splits, "fwd": "fa_fwd_splitkv (split forward + LSE merge, "
                            "both inside the fwd timing)"} if splits is not None else {}),
+                       **({"deterministic_bwd": "int64 fixed-point dQ accumulation"} if det else {}),
                        l2=f"inputs {in_bytes / 2**20:.0f} MiB per rank > 126 MiB L2, no flush"
                        if in_bytes > L2_BYTES else "inputs fit in L2"),
         "fwd_tflops": fwd_tflops, "fwd_ms": fwd_ms, "bwd_main_tflops": bmain_tflops, "bwd_main_ms": bmain_ms,
@@ -452,6 +456,8 @@ def main():
     ap.add_argument("--fwd-splits", type=int, default=None,
                     help="forward through fa_fwd_splitkv with this many key ranges (0: chosen for the "
                          "GPU; default: the workload's own setting)")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="backward in deterministic mode (bitwise repeatable dQ)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

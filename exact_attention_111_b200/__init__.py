@@ -3,7 +3,7 @@
 The binding marshals arguments only; every step of the computation runs in the CUDA
 kernels behind the C ABI of ``include/fa.h``.  The C entry points are mirrored one to one
 (``fa_fwd``, ``fa_bwd``, ``fa_fwd_ex``, ``fa_bwd_ex``, ``fa_bwd_workspace_bytes``,
-``fa_bwd_noalloc``, ``fa_fwd_partial``, ``fa_lse_merge``, ``fa_fwd_splitkv``,
+``fa_bwd_workspace_bytes_ex``, ``fa_bwd_noalloc``, ``fa_fwd_partial``, ``fa_lse_merge``, ``fa_fwd_splitkv``,
 ``fa_fwd_splitkv_workspace_bytes``, ``fa_splitkv_choose``, ``fa_check_status``,
 ``fa_status_string``, ``fa_last_launch_count``); they take torch tensors (or raw device
 addresses as ints).  ``attention_forward`` / ``attention_backward`` /
@@ -24,10 +24,10 @@ __all__ = [
     "attention_forward", "attention_backward", "FlashAttention", "FA_BF16", "FA_FP16", "FA_FP32",
     "fa_fwd_partial", "fa_lse_merge", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes",
     "fa_splitkv_choose", "attention_forward_splitkv", "attention_forward_partial", "lse_merge",
-    "FA_MAX_PARTS",
+    "FA_MAX_PARTS", "fa_bwd_workspace_bytes_ex", "FA_ERR_RANGE",
 ]
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE, FA_ERR_RANGE = range(7)
 FA_BF16, FA_FP16, FA_FP32 = 0, 1, 2
 TILE = 128
 FA_MAX_PARTS = 64
@@ -56,7 +56,7 @@ class BwdArgs(ctypes.Structure):
                 ("B", _i), ("H", _i), ("N", _i), ("d", _i), ("scale", _f), ("causal", _i),
                 ("blockmask", _vp), ("dtype", _i), ("visit_log", _vp),
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("stream", _vp),
-                ("main_start_event", _vp), ("main_stop_event", _vp)]
+                ("main_start_event", _vp), ("main_stop_event", _vp), ("deterministic", _i)]
 
 
 class PartialArgs(ctypes.Structure):
@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_ex.restype = _i
     L.fa_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
     L.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+    L.fa_bwd_workspace_bytes_ex.argtypes = [_i, _i, _i, _i, _i]
+    L.fa_bwd_workspace_bytes_ex.restype = ctypes.c_size_t
     L.fa_check_status.argtypes = [_vp]
     L.fa_check_status.restype = _i
     L.fa_status_string.argtypes = [_i]
@@ -145,6 +147,10 @@ def fa_last_launch_count() -> int:
 
 def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
     return lib().fa_bwd_workspace_bytes(B, H, N, d)
+
+
+def fa_bwd_workspace_bytes_ex(B: int, H: int, N: int, d: int, deterministic: bool) -> int:
+    return lib().fa_bwd_workspace_bytes_ex(B, H, N, d, int(bool(deterministic)))
 
 
 def fa_check_status(stream=None):
@@ -220,11 +226,11 @@ def _event(e):
 
 def fa_bwd_ex(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal=False, blockmask=None,
               dtype=FA_BF16, visit_log=None, workspace=None, workspace_bytes=0, stream=None,
-              main_start_event=None, main_stop_event=None):
+              main_start_event=None, main_stop_event=None, deterministic=False):
     a = BwdArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
                 _ptr(dv), B, H, N, d, scale, int(bool(causal)), _ptr(blockmask), dtype,
                 _ptr(visit_log), _ptr(workspace), workspace_bytes, _stream(stream),
-                _event(main_start_event), _event(main_stop_event))
+                _event(main_start_event), _event(main_stop_event), int(bool(deterministic)))
     _check(lib().fa_bwd_ex(ctypes.byref(a)), "fa_bwd_ex")
 
 
@@ -315,20 +321,21 @@ def lse_merge(o_parts, lse_parts, out_dtype=None, stream=None):
 
 
 def attention_backward(q, k, v, o, lse, dout, causal=False, blockmask=None, scale=None,
-                       workspace=None, visit_log=None, stream=None):
-    """Returns (dQ, dK, dV) for the gradient ``dout`` of O."""
+                       workspace=None, visit_log=None, stream=None, deterministic=False):
+    """Returns (dQ, dK, dV) for the gradient ``dout`` of O.  ``deterministic``: bitwise
+    repeatable dQ through the int64 fixed-point accumulator (include/fa.h)."""
     import torch
     _check_qkv(q, k, v, o, dout)
     B, H, N, d = q.shape
     scale = (1.0 / d ** 0.5) if scale is None else scale
-    nbytes = fa_bwd_workspace_bytes(B, H, N, d)
+    nbytes = fa_bwd_workspace_bytes_ex(B, H, N, d, deterministic)
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
     fa_bwd_ex(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockmask,
-              _dtype_code(q), visit_log, workspace, workspace.numel(), stream)
+              _dtype_code(q), visit_log, workspace, workspace.numel(), stream, deterministic=deterministic)
     return dq, dk, dv
 
 

@@ -15,6 +15,11 @@
 //             partial of each step is added into the fp32 accumulator;
 //   bwd_post  dQ = 16-bit(scale * accumulator).
 //
+// Deterministic mode (dq_fix set): the dQ partials are added as int64 fixed point (2^-32
+// resolution) by 64-bit bulk reduce-adds.  Integer addition is associative, so the sum -- and
+// dQ -- is bitwise independent of the order in which CTAs finish; the float path's order-
+// dependent fp32 additions are the only non-repeatable step of the backward.
+//
 // bwd_main roles (320 threads): warps 0-7 two compute groups, one key row per thread (TMEM
 // lanes), each group owning half of the query columns and draining half of each dQ partial;
 // warp 8 TMA producer; warp 9 MMA issuer.
@@ -61,9 +66,17 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreArgs a) {
         acc = fmaf(of.x, df.x, acc);
         acc = fmaf(of.y, df.y, acc);
       }
-      float4* z = reinterpret_cast<float4*>(a.dq_acc + off);
-      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a.dq_fix == nullptr) {
+        float4* z = reinterpret_cast<float4*>(a.dq_acc + off);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    if (a.dq_fix != nullptr && active) {       // every row of the padded accumulator, 4 x 16 bytes
+      const long long tile = (long long)bh * (a.Np / 128) + i / 128;
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        *reinterpret_cast<longlong2*>(a.dq_fix + fix_index(tile, i & 127, g * 8 + 2 * t, D)) = make_longlong2(0, 0);
     }
 #pragma unroll
     for (int s = G / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s, G);
@@ -94,6 +107,28 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdPostArgs a) {
     w.z = pack2<kFp16>(y.x * a.scale, y.y * a.scale);
     w.w = pack2<kFp16>(y.z * a.scale, y.w * a.scale);
     reinterpret_cast<uint4*>(a.dq)[t] = w;
+  }
+}
+
+// Deterministic mode: dQ = 16-bit(scale * 2^-32 * int64 accumulator), one thread per row
+// and 8 columns (four 16-byte pieces of the tile-blocked layout).
+template <int D, bool kFp16>
+__global__ void __launch_bounds__(256) bwd_post_fix_kernel(const BwdPostArgs a) {
+  constexpr int G = D / 8;
+  const long long total = (long long)a.BH * a.N * G;
+  const float f = a.scale * (1.0f / kFixOne);
+  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += (long long)gridDim.x * blockDim.x) {
+    const long long r = t / G;
+    const int g = (int)(t - r * G);
+    const int bh = (int)(r / a.N), i = (int)(r % a.N);
+    const long long tile = (long long)bh * (a.Np / 128) + i / 128;
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const longlong2 x = *reinterpret_cast<const longlong2*>(a.dq_fix + fix_index(tile, i & 127, g * 8 + 2 * u, D));
+      w[u] = pack2<kFp16>(__ll2float_rn(x.x) * f, __ll2float_rn(x.y) * f);
+    }
+    reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.dq) + r * D)[g] = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -160,7 +195,7 @@ __device__ __forceinline__ int next_kept(int k, int j, int T, int causal, const 
   return k;
 }
 
-template <int D, bool kFp16>
+template <int D, bool kFp16, bool kDet>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -386,6 +421,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int cc = 0; cc < kHalfD; cc += 32) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&v[cc]));
       tc_fence_before();
       mbar_arrive(&sh.dq_empty);                    // TMEM columns free for the next MMA
+      if constexpr (kDet) {
+        // int64 fixed point, 16 columns per bulk add: the warp's 32 rows x 16 columns are one
+        // contiguous 4 KB block of the accumulator (fix_index), staged as [pair][lane][2].
+        float mx = 0.f;
+#pragma unroll
+        for (int t = 0; t < kHalfD; ++t) mx = fmaxf(mx, fabsf(__uint_as_float(v[t])));
+        if (!(mx < kFixLimit)) atomicCAS(a.status, 0, kDevRange);   // also catches NaN
+        const long long tile = (long long)bh * a.T + ip;
+#pragma unroll
+        for (int ck = 0; ck < kHalfD / 16; ++ck) {
+          wait_stage_read();
+#pragma unroll
+          for (int pr = 0; pr < 8; ++pr) {
+            const long long x0 = __float2ll_rn(__uint_as_float(v[16 * ck + 2 * pr]) * kFixOne);
+            const long long x1 = __float2ll_rn(__uint_as_float(v[16 * ck + 2 * pr + 1]) * kFixOne);
+            *reinterpret_cast<longlong2*>(stage + pr * 512 + lane * 16) = make_longlong2(x0, x1);
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int col0 = kHalfD * g + 16 * ck;
+            bulk_reduce_add_u64(a.dq_fix + fix_index(tile, wq * 32, col0, D), stage, 4096);
+            bulk_commit();
+          }
+        }
+        return true;
+      }
 #pragma unroll
       for (int rd = 0; rd < kHalfD / 32; ++rd) {
         wait_stage_read();                          // previous reduce finished reading `stage`
@@ -549,7 +611,7 @@ template <int D, bool kFp16>
 cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                          const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t s) {
   using C = BwdCfg<D>;
-  auto kern = bwd_kernel<D, kFp16>;
+  auto kern = a.dq_fix != nullptr ? bwd_kernel<D, kFp16, true> : bwd_kernel<D, kFp16, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.T);
@@ -590,6 +652,16 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 
 cudaError_t launch_bwd_post(const BwdPostArgs& a, bool fp16, cudaStream_t s) {
   const int g = grid_for(a.n_elems / 8, 256);
+  if (a.dq_fix != nullptr) {
+    if (a.d == 64) {
+      if (fp16) bwd_post_fix_kernel<64, true><<<g, 256, 0, s>>>(a);
+      else bwd_post_fix_kernel<64, false><<<g, 256, 0, s>>>(a);
+    } else {
+      if (fp16) bwd_post_fix_kernel<128, true><<<g, 256, 0, s>>>(a);
+      else bwd_post_fix_kernel<128, false><<<g, 256, 0, s>>>(a);
+    }
+    return cudaGetLastError();
+  }
   if (fp16) bwd_post_kernel<true><<<g, 256, 0, s>>>(a);
   else bwd_post_kernel<false><<<g, 256, 0, s>>>(a);
   return cudaGetLastError();

@@ -125,12 +125,14 @@ struct WsLayout {
   size_t dq_acc, delta, lse2, total;
 };
 
-WsLayout ws_layout(int B, int H, int N, int d) {
+// The dQ accumulator is fp32 [BH, N, d], or in deterministic mode int64 over whole tiles
+// [BH, Np, d] (tile-blocked, fix_index).
+WsLayout ws_layout(int B, int H, int N, int d, bool det = false) {
   const size_t BH = (size_t)B * H;
   const size_t Np = (size_t)((N + kTile - 1) / kTile) * kTile;
   WsLayout w;
   w.dq_acc = 0;
-  w.delta = align256(BH * N * d * 4);
+  w.delta = det ? align256(BH * Np * d * 8) : align256(BH * N * d * 4);
   w.lse2 = w.delta + align256(BH * Np * 4);
   w.total = w.lse2 + align256(BH * Np * 4);
   return w;
@@ -170,6 +172,7 @@ const char* fa_status_string(int s) {
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_RANGE: return "FA_ERR_RANGE";
     default: return "FA_ERR_UNKNOWN";
   }
 }
@@ -179,6 +182,11 @@ int fa_last_launch_count(void) { return t_last_launches; }
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d, 1.f, FA_BF16) != FA_OK) return 0;
   return ws_layout(B, H, N, d).total;
+}
+
+size_t fa_bwd_workspace_bytes_ex(int B, int H, int N, int d, int deterministic) {
+  if (check_shape(B, H, N, d, 1.f, FA_BF16) != FA_OK) return 0;
+  return ws_layout(B, H, N, d, deterministic != 0).total;
 }
 
 int fa_fwd_ex(const fa_fwd_args* p) {
@@ -236,7 +244,8 @@ int fa_bwd_ex(const fa_bwd_args* p) {
       !aligned(x.dq, 16) || !aligned(x.dk, 16) || !aligned(x.dv, 16) || !aligned(x.lse, 4) ||
       !aligned(x.visit_log, 4))
     return FA_ERR_INVALID_ARG;
-  const WsLayout w = ws_layout(x.B, x.H, x.N, x.d);
+  const bool det = x.deterministic != 0;
+  const WsLayout w = ws_layout(x.B, x.H, x.N, x.d, det);
   if (!x.workspace || !aligned(x.workspace, 256) || x.workspace_bytes < w.total) return FA_ERR_WORKSPACE;
   const bool fp16 = x.dtype == FA_FP16;
   const int BH = x.B * x.H;
@@ -249,6 +258,7 @@ int fa_bwd_ex(const fa_bwd_args* p) {
     return FA_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(x.workspace);
   float* dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
+  long long* dq_fix = det ? reinterpret_cast<long long*>(ws + w.dq_acc) : nullptr;
   CUtensorMap tdq;
   if (!encode_dqacc(&tdq, dq_acc, BH, x.N, x.d)) return FA_ERR_CUDA;
   float* delta = reinterpret_cast<float*>(ws + w.delta);
@@ -260,12 +270,12 @@ int fa_bwd_ex(const fa_bwd_args* p) {
 
   BwdPreArgs pre{};
   pre.o = x.o; pre.dout = x.dout; pre.lse = x.lse;
-  pre.delta = delta; pre.lse2 = lse2; pre.dq_acc = dq_acc;
+  pre.delta = delta; pre.lse2 = lse2; pre.dq_acc = dq_acc; pre.dq_fix = dq_fix;
   pre.N = x.N; pre.Np = Np; pre.BH = BH; pre.d = x.d;
   if (launch_bwd_pre(pre, fp16, s) != cudaSuccess) return FA_ERR_CUDA;
 
   BwdArgs b{};
-  b.delta = delta; b.lse2 = lse2; b.dq_acc = dq_acc; b.dk = x.dk; b.dv = x.dv;
+  b.delta = delta; b.lse2 = lse2; b.dq_acc = dq_acc; b.dq_fix = dq_fix; b.dk = x.dk; b.dv = x.dv;
   b.blockmask = x.blockmask; b.visit = x.visit_log; b.status = status; b.timeout_ns = kWaitLimitNs;
   b.N = x.N; b.Np = Np; b.BH = BH; b.T = T; b.causal = x.causal != 0;
   b.group_heads = group_heads_for(BH, T);
@@ -278,7 +288,8 @@ int fa_bwd_ex(const fa_bwd_args* p) {
     return FA_ERR_CUDA;
 
   BwdPostArgs post{};
-  post.dq_acc = dq_acc; post.dq = x.dq; post.n_elems = (long long)BH * x.N * x.d; post.scale = x.scale;
+  post.dq_acc = dq_acc; post.dq_fix = dq_fix; post.dq = x.dq; post.n_elems = (long long)BH * x.N * x.d;
+  post.N = x.N; post.Np = Np; post.BH = BH; post.d = x.d; post.scale = x.scale;
   if (launch_bwd_post(post, fp16, s) != cudaSuccess) return FA_ERR_CUDA;
   t_last_launches = 3;
   return FA_OK;
@@ -461,7 +472,7 @@ int fa_check_status(void* stream) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
-    return v == kDevTimeout ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+    return v == kDevTimeout ? FA_ERR_TIMEOUT : v == kDevRange ? FA_ERR_RANGE : FA_ERR_CUDA;
   }
   return FA_OK;
 }

@@ -12,7 +12,14 @@ constexpr int kTile = 128;          // rows per query tile and keys per key/valu
 constexpr int kMaxTiles = 2048;     // tile lists live in shared memory (N <= 2048 * 128)
 
 // Error codes a kernel can record in the device status word (read by fa_check_status).
-enum : int { kDevOk = 0, kDevTimeout = 4, kDevBadState = 6 };
+enum : int { kDevOk = 0, kDevTimeout = 4, kDevBadState = 6, kDevRange = 7 };
+
+// Deterministic backward: dQ partials are added as int64 fixed point with 32 fraction bits.
+// Integer addition is associative, so the sum does not depend on the order in which the
+// key-tile CTAs add their partials.  A partial of magnitude >= 2^20 is reported (kDevRange):
+// with at most 2^11 key tiles the sum then stays below 2^31, inside the int64 range.
+constexpr float kFixOne = 4294967296.0f;      // 2^32
+constexpr float kFixLimit = 1048576.0f;       // 2^20
 
 constexpr int kMaxParts = 64;       // most key splits / merged parts per call
 
@@ -48,7 +55,9 @@ struct BwdPreArgs {
   const float* lse;         // [BH, N]
   float* delta;             // [BH, Np]  -D_i = -sum_c dO_ic O_ic (0 on padding rows)
   float* lse2;              // [BH, Np]  -LSE_i * log2(e) (-inf on padding / empty rows)
-  float* dq_acc;            // [BH, N, d] fp32, zeroed here
+  float* dq_acc;            // [BH, N, d] fp32, zeroed here (when dq_fix is null)
+  long long* dq_fix;        // deterministic mode: int64 fixed-point accumulator (tile-blocked,
+                            // see fix_index), zeroed here; null otherwise
   int N, Np, BH, d;
 };
 
@@ -56,6 +65,7 @@ struct BwdArgs {
   const float* delta;       // [BH, Np]  -D
   const float* lse2;        // [BH, Np]  -LSE * log2(e)
   float* dq_acc;            // [BH, N, d]
+  long long* dq_fix;        // deterministic mode only: [BH, Np, d] int64, tile-blocked
   void* dk;                 // [BH, N, d] 16-bit
   void* dv;                 // [BH, N, d] 16-bit
   const uint8_t* blockmask;
@@ -71,10 +81,25 @@ struct BwdArgs {
 
 struct BwdPostArgs {
   const float* dq_acc;      // [BH, N, d]
+  const long long* dq_fix;  // deterministic mode: the int64 accumulator (else null)
   void* dq;                 // [BH, N, d] 16-bit
   long long n_elems;
+  int N, Np, BH, d;
   float scale;
 };
+
+// Element (row, col) of query tile `tile` in the int64 accumulator.  Each tile is 128 x d
+// values cut into blocks of 32 rows x 16 columns (one compute warp's rows, one 128-byte
+// column chunk); a block is 8 column pairs x 32 rows x 2 values, so a warp's block is one
+// contiguous 4 KB range that a single bulk reduce adds, and that the warp stages in shared
+// memory with conflict-free 16-byte stores (lane = row).
+#ifdef __CUDACC__
+__host__ __device__
+#endif
+inline long long fix_index(long long tile, int row, int col, int d) {
+  const int blk = (col >> 4) * 4 + (row >> 5);
+  return tile * 128LL * d + ((((long long)blk * 8 + ((col & 15) >> 1)) * 32 + (row & 31)) * 2 + (col & 1));
+}
 
 // Launchers (defined next to each kernel).  Return a cudaError_t.
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdArgs& a,
@@ -82,7 +107,7 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 cudaError_t launch_bwd_pre(const BwdPreArgs& a, bool fp16, cudaStream_t s);
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int d, bool fp16,
-                       cudaStream_t s);
+                       cudaStream_t s);   // deterministic when a.dq_fix is set
 cudaError_t launch_bwd_post(const BwdPostArgs& a, bool fp16, cudaStream_t s);
 cudaError_t launch_merge(const MergeArgs& a, int d, cudaStream_t s);
 

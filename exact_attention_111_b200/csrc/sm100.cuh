@@ -129,6 +129,14 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const 
                "r"(smem_addr(src)), "r"(x), "r"(y), "r"(z)
                : "memory");
 }
+// 1-D bulk reduce: global[gdst .. +bytes) += shared[ssrc .. +bytes) as 64-bit integers
+// (two's complement, so signed values add correctly).  Both addresses 16-byte aligned,
+// bytes a multiple of 16.
+__device__ __forceinline__ void bulk_reduce_add_u64(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.u64 [%0], [%1], %2;"
+               :: "l"(gdst), "r"(smem_addr(ssrc)), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the shared-memory source of every committed bulk group has been read.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

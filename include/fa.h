@@ -41,7 +41,9 @@ typedef enum {
   FA_ERR_UNSUPPORTED = 2,   /* d not in {64, 128}, dtype not bf16/fp16, N too large        */
   FA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (no device, launch error)  */
   FA_ERR_TIMEOUT = 4,       /* a kernel's bounded wait expired (reported by fa_check_status) */
-  FA_ERR_WORKSPACE = 5      /* workspace pointer NULL/misaligned or smaller than required   */
+  FA_ERR_WORKSPACE = 5,     /* workspace pointer NULL/misaligned or smaller than required   */
+  FA_ERR_RANGE = 6          /* deterministic backward: a dQ partial was non-finite or too
+                               large for the fixed-point accumulator (fa_check_status)       */
 } fa_status;
 
 typedef enum {
@@ -117,14 +119,35 @@ typedef struct {
   void* main_start_event;  /* NULL, or a cudaEvent_t recorded on `stream` right before the
                               fused main backward kernel (for per-kernel timing)       */
   void* main_stop_event;   /* NULL, or a cudaEvent_t recorded right after it           */
+  int deterministic;       /* nonzero: bitwise repeatable dQ (see below); the workspace
+                              must then hold fa_bwd_workspace_bytes_ex(..., 1) bytes    */
 } fa_bwd_args;
 
 int fa_fwd_ex(const fa_fwd_args* args);
 int fa_bwd_ex(const fa_bwd_args* args);
 
 /*
+ * Deterministic backward (fa_bwd_args.deterministic != 0).  "Exact and deterministic" is a
+ * property the FlashAttention-2 wiki claims ("性能与效率"); the forward has it as built, but
+ * the default backward adds each key tile's fp32 dQ partial into the accumulator in whatever
+ * order the CTAs finish, and fp32 addition is not associative.  This mode adds the partials
+ * as int64 fixed point with 32 fraction bits instead: integer addition is associative, so
+ * dQ (and dK, dV, which never depended on order) are bitwise identical from run to run.
+ *   - cost: an int64 accumulator (twice the bytes of the fp32 one) over whole 128-row tiles;
+ *   - precision: each partial is rounded to a multiple of 2^-32 before the (exact) sum, an
+ *     absolute error of at most T * 2^-33 on scale^-1 * dQ;
+ *   - range: a partial with magnitude >= 2^20 (or non-finite) makes the call report
+ *     FA_ERR_RANGE through fa_check_status; the sum of up to 2048 tiles then stays inside
+ *     the int64 range, so no result is silently wrapped.
+ * Workspace bytes for either mode; fa_bwd_workspace_bytes(...) == ..._ex(..., 0).
+ */
+size_t fa_bwd_workspace_bytes_ex(int B, int H, int N, int d, int deterministic);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that kernels set
- * when a bounded wait expires.  Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA.
+ * when a bounded wait expires (FA_ERR_TIMEOUT) or a deterministic backward meets a partial
+ * outside its range (FA_ERR_RANGE).  Returns FA_OK, FA_ERR_TIMEOUT, FA_ERR_RANGE or
+ * FA_ERR_CUDA.
  */
 int fa_check_status(void* stream);
 

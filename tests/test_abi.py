@@ -226,3 +226,25 @@ def test_merge_argument_errors(L):
     assert call(parts=[FAKE, None]) == fa.FA_ERR_INVALID_ARG
     assert call(parts=[FAKE, FAKE + 4]) == fa.FA_ERR_INVALID_ARG   # O part not 16-byte aligned
     assert call(o=None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_deterministic_workspace_formula(L):
+    # int64 accumulator over whole 128-row tiles, then the two fp32 row vectors
+    a = lambda x: (x + 255) // 256 * 256
+    for B, H, N, d in ((1, 1, 128, 64), (64, 16, 1024, 64), (2, 3, 1000, 128), (1, 1, 1, 64)):
+        Np = (N + 127) // 128 * 128
+        assert fa.fa_bwd_workspace_bytes_ex(B, H, N, d, True) == a(B * H * Np * d * 8) + 2 * a(B * H * Np * 4)
+        assert fa.fa_bwd_workspace_bytes_ex(B, H, N, d, False) == fa.fa_bwd_workspace_bytes(B, H, N, d)
+    assert fa.fa_bwd_workspace_bytes_ex(1, 1, 128, 96, True) == 0
+
+
+def test_deterministic_needs_its_workspace(L):
+    import ctypes as ct
+    ws_det = fa.fa_bwd_workspace_bytes_ex(1, 1, 1000, 64, True)
+    ws = fa.fa_bwd_workspace_bytes(1, 1, 1000, 64)
+    p = FAKE
+    a = fa.BwdArgs(p, p, p, p, p, p, p, p, p, 1, 1, 1000, 64, 0.125, 0, None, fa.FA_BF16, None,
+                   0x100000, ws_det - 1, None, None, None, 1)
+    assert L.fa_bwd_ex(ct.byref(a)) == fa.FA_ERR_WORKSPACE
+    assert ws < ws_det
+    assert fa.fa_status_string(fa.FA_ERR_RANGE) == "FA_ERR_RANGE"
