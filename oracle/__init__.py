@@ -11,3 +11,11 @@ from .attention import (  # noqa: F401
     lse_merge,
     softmax_rows,
 )
+from .dropout import (  # noqa: F401
+    attention_bwd_dropout,
+    attention_fwd_dropout,
+    drop_threshold,
+    keep_mask,
+    keep_scale,
+    philox4x32_10,
+)
