@@ -270,8 +270,15 @@ def run_ours(args, w, world, rank, local):
         wsfb = fa.fa_fwd_splitkv_workspace_bytes(B, H, N, D, splits)
         wsf = torch.empty(wsfb, dtype=torch.uint8, device=dev)
 
+    pdrop, dseed = float(args.dropout), 0x5EED
+    if pdrop > 0 and splits is not None:
+        raise SystemExit("--dropout does not combine with the split-KV forward")
+
     def forward(q, k, v, o_, lse_):
-        if splits is None:
+        if pdrop > 0:
+            fa.fa_fwd_ex(q, k, v, o_, lse_, B, H, N, D, scale, w.causal, mask, fa.FA_BF16, False, None, stream,
+                         dropout_p=pdrop, dropout_seed=dseed)
+        elif splits is None:
             fa.fa_fwd(q, k, v, o_, lse_, B, H, N, D, scale, w.causal, mask, stream)
         else:
             fa.fa_fwd_splitkv(q, k, v, o_, lse_, B, H, N, D, scale, w.causal, mask, splits, wsf, wsfb, stream)
@@ -292,7 +299,7 @@ def run_ours(args, w, world, rank, local):
         fa.fa_bwd_ex(d["q"], d["k"], d["v"], o, lse, d["dout"], dq, dk, dv, B, H, N, D, scale, w.causal, mask,
                      fa.FA_BF16, None, ws, wsb, stream,
                      timed_kernels["b0"] if timed_kernels else None, timed_kernels["b1"] if timed_kernels else None,
-                     deterministic=det)
+                     deterministic=det, dropout_p=pdrop, dropout_seed=dseed)
         launches[0] += fa.fa_last_launch_count()
 
     # ---------------------------------------------------------------- warm-up
@@ -378,7 +385,7 @@ def run_ours(args, w, world, rank, local):
             forward(din["q"], din["k"], din["v"], dres["o"], dres["lse"])
             fa.fa_bwd_ex(din["q"], din["k"], din["v"], dres["o"], dres["lse"], din["dout"], dres["dq"], dres["dk"],
                          dres["dv"], B, H, N, D, scale, w.causal, mask, fa.FA_BF16, None, ws, wsb, stream,
-                         deterministic=det)
+                         deterministic=det, dropout_p=pdrop, dropout_seed=dseed)
             ev_comp[b].record(stream)
             s_down.wait_event(ev_comp[b])
             with torch.cuda.stream(s_down):
@@ -410,7 +417,7 @@ def run_ours(args, w, world, rank, local):
         dom, dom_tf, dom_flops = "bwd_main", bmain_tflops, bwd_flops
     else:
         dom, dom_tf, dom_flops = "fwd", fwd_tflops, fwd_flops
-    traffic = stored_traffic(dom, w.name) if not det else None   # captured for the default mode only
+    traffic = stored_traffic(dom, w.name) if not (det or pdrop > 0) else None   # captured for the default mode only
     roofline = {"bound": "tensor", "achieved": dom_tf, "peak": peak_sust, "unit": "TFLOP/s",
                 "frac": dom_tf / peak_sust, "traffic": traffic, "kernel": dom,
                 "peak_source": f"bf16_tflops_sustained of {peak_src} (MEASURED_PEAKS.json)",
@@ -424,6 +431,8 @@ def run_ours(args, w, world, rank, local):
                        **({"fwd_splits": splits, "fwd": "fa_fwd_splitkv (split forward + LSE merge, "
                            "both inside the fwd timing)"} if splits is not None else {}),
                        **({"deterministic_bwd": "int64 fixed-point dQ accumulation"} if det else {}),
+                       **({"dropout_p": pdrop, "dropout": "fused, Philox4x32-10 mask regenerated in the backward"}
+                          if pdrop > 0 else {}),
                        l2=f"inputs {in_bytes / 2**20:.0f} MiB per rank > 126 MiB L2, no flush"
                        if in_bytes > L2_BYTES else "inputs fit in L2"),
         "fwd_tflops": fwd_tflops, "fwd_ms": fwd_ms, "bwd_main_tflops": bmain_tflops, "bwd_main_ms": bmain_ms,
@@ -456,6 +465,8 @@ def main():
     ap.add_argument("--fwd-splits", type=int, default=None,
                     help="forward through fa_fwd_splitkv with this many key ranges (0: chosen for the "
                          "GPU; default: the workload's own setting)")
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="fused dropout probability in both passes (default 0: none)")
     ap.add_argument("--deterministic", action="store_true",
                     help="backward in deterministic mode (bitwise repeatable dQ)")
     args = ap.parse_args()

@@ -46,7 +46,7 @@ class FwdArgs(ctypes.Structure):
     _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("o", _vp), ("lse", _vp),
                 ("B", _i), ("H", _i), ("N", _i), ("d", _i), ("scale", _f), ("causal", _i),
                 ("blockmask", _vp), ("dtype", _i), ("o_fp32", _i), ("visit_log", _vp),
-                ("stream", _vp)]
+                ("stream", _vp), ("dropout_p", _f), ("dropout_seed", ctypes.c_ulonglong)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -56,7 +56,8 @@ class BwdArgs(ctypes.Structure):
                 ("B", _i), ("H", _i), ("N", _i), ("d", _i), ("scale", _f), ("causal", _i),
                 ("blockmask", _vp), ("dtype", _i), ("visit_log", _vp),
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("stream", _vp),
-                ("main_start_event", _vp), ("main_stop_event", _vp), ("deterministic", _i)]
+                ("main_start_event", _vp), ("main_stop_event", _vp), ("deterministic", _i),
+                ("dropout_p", _f), ("dropout_seed", ctypes.c_ulonglong)]
 
 
 class PartialArgs(ctypes.Structure):
@@ -179,9 +180,10 @@ def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
 
 
 def fa_fwd_ex(q, k, v, o, lse, B, H, N, d, scale, causal=False, blockmask=None, dtype=FA_BF16,
-              o_fp32=False, visit_log=None, stream=None):
+              o_fp32=False, visit_log=None, stream=None, dropout_p=0.0, dropout_seed=0):
     a = FwdArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale, int(bool(causal)),
-                _ptr(blockmask), dtype, int(bool(o_fp32)), _ptr(visit_log), _stream(stream))
+                _ptr(blockmask), dtype, int(bool(o_fp32)), _ptr(visit_log), _stream(stream),
+                float(dropout_p), int(dropout_seed))
     _check(lib().fa_fwd_ex(ctypes.byref(a)), "fa_fwd_ex")
 
 
@@ -226,11 +228,12 @@ def _event(e):
 
 def fa_bwd_ex(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal=False, blockmask=None,
               dtype=FA_BF16, visit_log=None, workspace=None, workspace_bytes=0, stream=None,
-              main_start_event=None, main_stop_event=None, deterministic=False):
+              main_start_event=None, main_stop_event=None, deterministic=False, dropout_p=0.0, dropout_seed=0):
     a = BwdArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
                 _ptr(dv), B, H, N, d, scale, int(bool(causal)), _ptr(blockmask), dtype,
                 _ptr(visit_log), _ptr(workspace), workspace_bytes, _stream(stream),
-                _event(main_start_event), _event(main_stop_event), int(bool(deterministic)))
+                _event(main_start_event), _event(main_stop_event), int(bool(deterministic)),
+                float(dropout_p), int(dropout_seed))
     _check(lib().fa_bwd_ex(ctypes.byref(a)), "fa_bwd_ex")
 
 
@@ -254,8 +257,9 @@ def _check_qkv(*ts):
 
 
 def attention_forward(q, k, v, causal=False, blockmask=None, scale=None, o_fp32=False,
-                      visit_log=None, stream=None):
-    """Returns (O, LSE) for [B, H, N, d] CUDA tensors (bf16 or fp16)."""
+                      visit_log=None, stream=None, dropout_p=0.0, dropout_seed=0):
+    """Returns (O, LSE) for [B, H, N, d] CUDA tensors (bf16 or fp16).  ``dropout_p`` > 0 drops
+    probabilities with the Philox mask of ``dropout_seed`` (include/fa.h)."""
     import torch
     _check_qkv(q, k, v)
     B, H, N, d = q.shape
@@ -263,7 +267,7 @@ def attention_forward(q, k, v, causal=False, blockmask=None, scale=None, o_fp32=
     o = torch.empty(q.shape, dtype=torch.float32 if o_fp32 else q.dtype, device=q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     fa_fwd_ex(q, k, v, o, lse, B, H, N, d, scale, causal, blockmask, _dtype_code(q), o_fp32,
-              visit_log, stream)
+              visit_log, stream, dropout_p=dropout_p, dropout_seed=dropout_seed)
     return o, lse
 
 
@@ -321,7 +325,8 @@ def lse_merge(o_parts, lse_parts, out_dtype=None, stream=None):
 
 
 def attention_backward(q, k, v, o, lse, dout, causal=False, blockmask=None, scale=None,
-                       workspace=None, visit_log=None, stream=None, deterministic=False):
+                       workspace=None, visit_log=None, stream=None, deterministic=False, dropout_p=0.0,
+                       dropout_seed=0):
     """Returns (dQ, dK, dV) for the gradient ``dout`` of O.  ``deterministic``: bitwise
     repeatable dQ through the int64 fixed-point accumulator (include/fa.h)."""
     import torch
@@ -335,7 +340,8 @@ def attention_backward(q, k, v, o, lse, dout, causal=False, blockmask=None, scal
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
     fa_bwd_ex(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockmask,
-              _dtype_code(q), visit_log, workspace, workspace.numel(), stream, deterministic=deterministic)
+              _dtype_code(q), visit_log, workspace, workspace.numel(), stream, deterministic=deterministic,
+              dropout_p=dropout_p, dropout_seed=dropout_seed)
     return dq, dk, dv
 
 

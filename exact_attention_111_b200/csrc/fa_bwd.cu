@@ -15,6 +15,13 @@
 //             partial of each step is added into the fp32 accumulator;
 //   bwd_post  dQ = 16-bit(scale * accumulator).
 //
+// Dropout (kDrop): the mask of the forward pass is regenerated from the same Philox4x32-10
+// counters ("核心方法 / Backward recomputation" regenerates it from the generator state):
+// dV = (P o M)ᵀ dO, and dS = P o (dP o M - D).  A compute thread owns one key row and 64 query
+// columns, while one generator call covers 16 keys of one query row, so each warp draws its
+// 128 calls (64 columns x 2 blocks of 16 keys) four per lane and hands each key row its bytes
+// with 64 shuffles (see drop_bits).
+//
 // Deterministic mode (dq_fix set): the dQ partials are added as int64 fixed point (2^-32
 // resolution) by 64-bit bulk reduce-adds.  Integer addition is associative, so the sum -- and
 // dQ -- is bitwise independent of the order in which CTAs finish; the float path's order-
@@ -184,6 +191,46 @@ __device__ __forceinline__ int rot_tile(int k, int j, int T) {
   return i < T ? i : i - T;
 }
 
+// Keep bits of the 64 query columns q0 .. q0+63 for this lane's key row (32 * wq + lane of key
+// tile j): bit c of the result is the decision for query q0 + c.
+// Lane L draws the calls of columns 4 * (L % 16) + k (k = 0..3) for the key block of its
+// half-warp, and stores each call's words rotated by L % 4.  Then in round (k, q, s) a lane
+// of word group w = (L % 16) / 4 reads slot s from lane 16 * half + 4q + ((w - s) mod 4),
+// which holds word w there: 64 shuffles deliver each lane the byte of all 64 columns.
+__device__ __forceinline__ uint64_t drop_bits(const Dropout& dr, int j, int wq, int lane, int q0, int bh) {
+  const int half = lane >> 4;
+  const uint32_t jb = static_cast<uint32_t>((j * kTile + wq * 32) >> 4) + half;
+  const int rot = lane & 3;
+  uint32_t R[4][4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint4 w4 = philox4x32_10(make_uint4(jb, static_cast<uint32_t>(q0 + 4 * (lane & 15) + k),
+                                              static_cast<uint32_t>(bh), 0u), dr.seed_lo, dr.seed_hi);
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      const int idx = (sl + rot) & 3;
+      R[k][sl] = (idx & 2) ? ((idx & 1) ? w4.w : w4.z) : ((idx & 1) ? w4.y : w4.x);
+    }
+  }
+  const int w = (lane & 15) >> 2;
+  const int bsh = 8 * (lane & 3);
+  uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int sl = 0; sl < 4; ++sl) {
+        const int g4 = (w - sl) & 3;
+        const uint32_t x = __shfl_sync(0xffffffffu, R[k][sl], (half << 4) | (4 * q + g4));
+        const uint32_t bit = ((x >> bsh) & 0xFFu) >= dr.t ? 1u : 0u;
+        const int cpos = (16 * q + 4 * g4 + k) & 31;
+        if (q < 2) lo |= bit << cpos;
+        else hi |= bit << cpos;
+      }
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 // Next step k' >= k whose query tile the key tile j keeps (T when none).
 __device__ __forceinline__ int next_kept(int k, int j, int T, int causal, const uint8_t* mask) {
   for (; k < T; ++k) {
@@ -195,7 +242,7 @@ __device__ __forceinline__ int next_kept(int k, int j, int T, int causal, const 
   return k;
 }
 
-template <int D, bool kFp16, bool kDet>
+template <int D, bool kFp16, bool kDet, bool kDrop>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -446,23 +493,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bulk_commit();
           }
         }
-        return true;
-      }
+      } else {
 #pragma unroll
-      for (int rd = 0; rd < kHalfD / 32; ++rd) {
-        wait_stage_read();                          // previous reduce finished reading `stage`
-        uint8_t* row_base = stage + lane * 128;
+        for (int rd = 0; rd < kHalfD / 32; ++rd) {
+          wait_stage_read();                          // previous reduce finished reading `stage`
+          uint8_t* row_base = stage + lane * 128;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const int phys = ch ^ (lane & 7);
-          *reinterpret_cast<uint4*>(row_base + phys * 16) =
-              make_uint4(v[32 * rd + 4 * ch], v[32 * rd + 4 * ch + 1], v[32 * rd + 4 * ch + 2], v[32 * rd + 4 * ch + 3]);
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_reduce_add_3d(&tm_dq, stage, kHalfD * g + 32 * rd, ip * kTile + wq * 32, bh);
-          bulk_commit();
+          for (int ch = 0; ch < 8; ++ch) {
+            const int phys = ch ^ (lane & 7);
+            *reinterpret_cast<uint4*>(row_base + phys * 16) =
+                make_uint4(v[32 * rd + 4 * ch], v[32 * rd + 4 * ch + 1], v[32 * rd + 4 * ch + 2], v[32 * rd + 4 * ch + 3]);
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_3d(&tm_dq, stage, kHalfD * g + 32 * rd, ip * kTile + wq * 32, bh);
+            bulk_commit();
+          }
         }
       }
       return true;
@@ -471,6 +518,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int k = k_first; k < a.T; k = next_kept(k + 1, j, a.T, a.causal, a.blockmask), ++c) {
         const int i = rot_tile(k, j, a.T);
         const int s = c % C::kStages;
+        uint32_t keep_lo = 0u, keep_hi = 0u;        // dropout keep bits of this row's 64 columns
+        if constexpr (kDrop) {
+          const uint64_t kb = drop_bits(a.drop, j, wq, lane, i * kTile + 64 * g, bh);
+          keep_lo = static_cast<uint32_t>(kb);
+          keep_hi = static_cast<uint32_t>(kb >> 32);
+        }
         ok = mbar_wait(&sh.q_full[s], (c / C::kStages) & 1, abort_flag, st) &&
              mbar_wait(&sh.s_full, c & 1, abort_flag, st);
         if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
@@ -514,7 +567,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // Pᵀ of this group's 64 query columns, packed two per 32-bit column, goes over the
         // first half of the group's own Sᵀ columns [64g, 64g+32): the other group may still be
         // reading its Sᵀ columns, so neither group writes outside its own range.
-        tmem_st32(tS + 64 * g, pk);
+        if constexpr (kDrop) {
+          // dV takes P o M: dropped columns 0, kept ones scaled (pk keeps the undropped P)
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t pd[16];
+            const uint32_t kw = h2 == 0 ? keep_lo : keep_hi;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              const float2 p = unpack2<kFp16>(pk[16 * h2 + t]);
+              pd[t] = pack2<kFp16>(((kw >> (2 * t)) & 1u) ? p.x * a.drop.scale : 0.f,
+                                   ((kw >> (2 * t + 1)) & 1u) ? p.y * a.drop.scale : 0.f);
+            }
+            tmem_st16(tS + 64 * g + 16 * h2, pd);
+          }
+        } else {
+          tmem_st32(tS + 64 * g, pk);
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sh.p_full);
@@ -543,7 +612,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int hh = 0; hh < 2; ++hh) {
               const int t = 2 * t4 + hh;                // pair index within the group's 64 columns
               const float2 p = unpack2<kFp16>(pk[t]);
-              const float2 dp = make_float2(__uint_as_float(dpv[2 * t]), __uint_as_float(dpv[2 * t + 1]));
+              float2 dp = make_float2(__uint_as_float(dpv[2 * t]), __uint_as_float(dpv[2 * t + 1]));
+              if constexpr (kDrop) {                    // dP o M
+                const uint32_t kw = t < 16 ? keep_lo : keep_hi;
+                dp.x = ((kw >> ((2 * t) & 31)) & 1u) ? dp.x * a.drop.scale : 0.f;
+                dp.y = ((kw >> ((2 * t + 1) & 31)) & 1u) ? dp.y * a.drop.scale : 0.f;
+              }
               const float2 ds = mul2(p, add2(dp, hh == 0 ? make_float2(nd.x, nd.y) : make_float2(nd.z, nd.w)));
               w[t] = pack2<kFp16>(ds.x, ds.y);
             }
@@ -611,7 +685,9 @@ template <int D, bool kFp16>
 cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                          const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t s) {
   using C = BwdCfg<D>;
-  auto kern = a.dq_fix != nullptr ? bwd_kernel<D, kFp16, true> : bwd_kernel<D, kFp16, false>;
+  const bool drop = a.drop.t > 0;
+  auto kern = a.dq_fix != nullptr ? (drop ? bwd_kernel<D, kFp16, true, true> : bwd_kernel<D, kFp16, true, false>)
+                                  : (drop ? bwd_kernel<D, kFp16, false, true> : bwd_kernel<D, kFp16, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.T);

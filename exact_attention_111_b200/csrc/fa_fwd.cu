@@ -30,6 +30,11 @@
 // split_tiles tiles, one CTA per (query pair, range), when there are too few query tiles to
 // fill the GPU.  Each range then writes its own normalised O and LSE (fp32) for a separate
 // merge kernel to combine; causal and block masks compare query-sequence positions.
+//
+// Dropout (kDrop, "核心方法 / Kernel fusion"): the softmax thread of row i draws the bytes
+// of its scores from Philox4x32-10, one call per 16 keys (counter (key / 16, i, bh, 0)), and
+// writes P o M (M = keep * 256/(256 - t)) to TMEM for the PV product, while the row max,
+// exp-sum and LSE stay those of the undropped P.
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -61,7 +66,7 @@ struct FwdShared {
 
 constexpr float kLn2 = 0.693147180559945309f;
 
-template <int D, bool kFp16>
+template <int D, bool kFp16, bool kDrop>
 __global__ void __launch_bounds__(320, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
@@ -300,13 +305,28 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         uint32_t pk[16];
+        uint4 rnd = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
+          if constexpr (kDrop) {
+            // keys kpos0 + 32h + 2i, +1 lie in 16-key block kpos0/16 + 2h + i/8, bytes 2(i%8), +1
+            if ((i & 7) == 0)
+              rnd = philox4x32_10(make_uint4(static_cast<uint32_t>(kpos0 >> 4) + 2 * h + (i >> 3),
+                                             static_cast<uint32_t>(row), static_cast<uint32_t>(bh), 0u),
+                                  a.drop.seed_lo, a.drop.seed_hi);
+          }
           const float2 t = fma2(make_float2(s[32 * h + 2 * i], s[32 * h + 2 * i + 1]), sl2v, mnegv);
           // kPolyOf8 of every 8 pairs go to the FMA-pipe polynomial, the rest to the SFU
           const float2 p = (((16 * h + i) & 7) < C::kPolyOf8) ? exp2_poly2(t) : make_float2(ex2(t.x), ex2(t.y));
           acc[i & 3] = add2(acc[i & 3], p);
-          pk[i] = pack2<kFp16>(p.x, p.y);
+          if constexpr (kDrop) {
+            const int wi = (i & 7) >> 1;
+            const uint32_t wv = wi == 0 ? rnd.x : wi == 1 ? rnd.y : wi == 2 ? rnd.z : rnd.w;
+            const uint32_t b0 = (wv >> (16 * (i & 1))) & 0xFFu, b1 = (wv >> (16 * (i & 1) + 8)) & 0xFFu;
+            pk[i] = pack2<kFp16>(b0 >= a.drop.t ? p.x * a.drop.scale : 0.f, b1 >= a.drop.t ? p.y * a.drop.scale : 0.f);
+          } else {
+            pk[i] = pack2<kFp16>(p.x, p.y);
+          }
         }
         tmem_st16(tS + 16 * h, pk);
       }
@@ -392,7 +412,7 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          cudaStream_t s) {
   using C = FwdCfg<D>;
   const size_t smem = C::kSmemTiles + (size_t)min(a.Tk, a.split_tiles) * sizeof(int) + 1024;
-  auto kern = fwd_kernel<D, kFp16>;
+  auto kern = a.drop.t > 0 ? fwd_kernel<D, kFp16, true> : fwd_kernel<D, kFp16, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.n_units) * static_cast<unsigned>(a.n_splits);

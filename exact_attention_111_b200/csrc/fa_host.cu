@@ -83,6 +83,18 @@ int check_shape(int B, int H, int N, int d, float scale, int dtype) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Dropout parameters: byte threshold t = floor(256 p + 1/2) (at most 255), scale 256/(256 - t).
+bool make_dropout(float p, unsigned long long seed, Dropout* d) {
+  if (!(p >= 0.f && p < 1.f)) return false;
+  int t = (int)std::floor(256.0 * (double)p + 0.5);
+  if (t > 255) t = 255;
+  d->t = (uint32_t)t;
+  d->scale = (float)(256.0 / (256.0 - t));
+  d->seed_lo = (uint32_t)(seed & 0xFFFFFFFFull);
+  d->seed_hi = (uint32_t)(seed >> 32);
+  return true;
+}
+
 // The forward's grid is BH x units x splits CTAs, indexed by an int.
 bool fwd_grid_ok(int BH, int units, int splits) {
   return (long long)BH * units * splits <= (long long)0x7fffffff;
@@ -198,6 +210,8 @@ int fa_fwd_ex(const fa_fwd_args* p) {
   if (!aligned(x.q, 16) || !aligned(x.k, 16) || !aligned(x.v, 16) || !aligned(x.o, 16) || !aligned(x.lse, 4) ||
       !aligned(x.visit_log, 4))
     return FA_ERR_INVALID_ARG;
+  Dropout drop{};
+  if (!make_dropout(x.dropout_p, x.dropout_seed, &drop)) return FA_ERR_INVALID_ARG;
   const bool fp16 = x.dtype == FA_FP16;
   const int BH = x.B * x.H;
   const int T = (x.N + kTile - 1) / kTile;
@@ -217,6 +231,7 @@ int fa_fwd_ex(const fa_fwd_args* p) {
   self_fwd_args(a, BH, x.N);
   a.causal = x.causal != 0;
   a.o_fp32 = x.o_fp32 != 0;
+  a.drop = drop;
   a.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
   t_last_launches = 0;
   if (launch_fwd(tq, tk, tv, a, x.d, fp16, static_cast<cudaStream_t>(x.stream)) != cudaSuccess) return FA_ERR_CUDA;
@@ -244,6 +259,8 @@ int fa_bwd_ex(const fa_bwd_args* p) {
       !aligned(x.dq, 16) || !aligned(x.dk, 16) || !aligned(x.dv, 16) || !aligned(x.lse, 4) ||
       !aligned(x.visit_log, 4))
     return FA_ERR_INVALID_ARG;
+  Dropout drop{};
+  if (!make_dropout(x.dropout_p, x.dropout_seed, &drop)) return FA_ERR_INVALID_ARG;
   const bool det = x.deterministic != 0;
   const WsLayout w = ws_layout(x.B, x.H, x.N, x.d, det);
   if (!x.workspace || !aligned(x.workspace, 256) || x.workspace_bytes < w.total) return FA_ERR_WORKSPACE;
@@ -281,6 +298,7 @@ int fa_bwd_ex(const fa_bwd_args* p) {
   b.group_heads = group_heads_for(BH, T);
   b.scale = x.scale;
   b.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
+  b.drop = drop;
   if (x.main_start_event && cudaEventRecord(static_cast<cudaEvent_t>(x.main_start_event), s) != cudaSuccess)
     return FA_ERR_CUDA;
   if (launch_bwd(tq, tk, tv, tdo, tdq, b, x.d, fp16, s) != cudaSuccess) return FA_ERR_CUDA;

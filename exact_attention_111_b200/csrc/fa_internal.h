@@ -23,6 +23,16 @@ constexpr float kFixLimit = 1048576.0f;       // 2^20
 
 constexpr int kMaxParts = 64;       // most key splits / merged parts per call
 
+// Dropout on the probabilities (off when t == 0).  Score (i, j) of head index bh is dropped
+// iff byte j mod 16 of Philox4x32-10(counter (j / 16, i, bh, 0), key (seed_lo, seed_hi)) is
+// below t (bytes little-endian within the four output words); kept scores are multiplied
+// by scale = 256 / (256 - t).
+struct Dropout {
+  uint32_t t;
+  float scale;
+  uint32_t seed_lo, seed_hi;
+};
+
 struct FwdArgs {
   void* o;                  // [BH, N, d] 16-bit, or fp32 when o_fp32 (split s at o + s * o_split_stride)
   float* lse;               // [BH, N]                                (split s at lse + s * lse_split_stride)
@@ -38,6 +48,7 @@ struct FwdArgs {
   int group_heads;          // CTAs are ordered in groups of this many heads (see cta_order)
   int causal, o_fp32;
   float scale_log2;         // scale * log2(e)
+  Dropout drop;
 };
 
 struct MergeArgs {
@@ -77,6 +88,7 @@ struct BwdArgs {
   int causal;
   float scale;              // multiplies dK (dQ is scaled in the post pass)
   float scale_log2;
+  Dropout drop;
 };
 
 struct BwdPostArgs {

@@ -103,6 +103,8 @@ typedef struct {
   int* visit_log;          /* NULL, or device int32 [B, H, T, T] that the kernel
                               increments once per (query tile, key tile) it computes */
   void* stream;
+  float dropout_p;         /* 0 (off) or a dropout probability in [0, 1), see below  */
+  unsigned long long dropout_seed;
 } fa_fwd_args;
 
 typedef struct {
@@ -121,10 +123,28 @@ typedef struct {
   void* main_stop_event;   /* NULL, or a cudaEvent_t recorded right after it           */
   int deterministic;       /* nonzero: bitwise repeatable dQ (see below); the workspace
                               must then hold fa_bwd_workspace_bytes_ex(..., 1) bytes    */
+  float dropout_p;         /* exactly the forward's dropout_p and dropout_seed        */
+  unsigned long long dropout_seed;
 } fa_bwd_args;
 
 int fa_fwd_ex(const fa_fwd_args* args);
 int fa_bwd_ex(const fa_bwd_args* args);
+
+/*
+ * Dropout on the attention probabilities, fused into both passes (FlashAttention-NeurIPS22
+ * summary, "核心方法 / Kernel fusion"; the backward regenerates the mask from the generator
+ * state instead of storing it, "Backward recomputation").  With dropout_p > 0:
+ *   - score (i, j) of head (b, h) draws byte (j mod 16) of Philox4x32-10 (Salmon et al.,
+ *     SC'11) at counter (j / 16, i, b * H + h, 0) with key (seed mod 2^32, seed / 2^32),
+ *     bytes little-endian within the four 32-bit output words;
+ *   - it is dropped iff that byte < t = floor(256 * dropout_p + 1/2) (at most 255), so the
+ *     probability is applied in steps of 1/256; kept probabilities are scaled by
+ *     256 / (256 - t), so the mask has mean exactly 1;
+ *   - O = (P o M) V, while LSE stays the log-sum-exp of the undropped scores;
+ *   - the backward must get the same dropout_p and dropout_seed as the forward.
+ * dropout_p outside [0, 1) (or NaN) returns FA_ERR_INVALID_ARG.  A value small enough that
+ * t = 0 means no dropout.  The split-KV and key-slice entry points take no dropout.
+ */
 
 /*
  * Deterministic backward (fa_bwd_args.deterministic != 0).  "Exact and deterministic" is a

@@ -248,3 +248,14 @@ def test_deterministic_needs_its_workspace(L):
     assert L.fa_bwd_ex(ct.byref(a)) == fa.FA_ERR_WORKSPACE
     assert ws < ws_det
     assert fa.fa_status_string(fa.FA_ERR_RANGE) == "FA_ERR_RANGE"
+
+
+def test_dropout_argument_errors(L):
+    import ctypes as ct
+    for p in (1.0, -0.1, float("nan"), 2.0):
+        a = fa.FwdArgs(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None, fa.FA_BF16, 0, None, None, p, 1)
+        assert L.fa_fwd_ex(ct.byref(a)) == fa.FA_ERR_INVALID_ARG, p
+        ws = fa.fa_bwd_workspace_bytes(1, 1, 128, 64)
+        b = fa.BwdArgs(*([FAKE] * 9), 1, 1, 128, 64, 0.125, 0, None, fa.FA_BF16, None, 0x100000, ws, None, None, None,
+                       0, p, 1)
+        assert L.fa_bwd_ex(ct.byref(b)) == fa.FA_ERR_INVALID_ARG, p

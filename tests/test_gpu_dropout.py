@@ -1,0 +1,155 @@
+"""GPU: fused dropout in the forward and backward kernels against the fp64 dropout oracle
+(oracle/dropout.py: Philox4x32-10 mask, byte threshold t = round(256 p), scale 256/(256-t)).
+
+O tolerance: the only arithmetic that changes against the plain forward is that the 16-bit
+PV operand is P * 256/(256 - t) instead of P, so its rounding error -- the term the 1e-2
+O bound absorbs (the oracle does not round P) -- grows by that factor; the bound is
+1e-2 * 256/(256 - t).  LSE (undropped) and the gradients keep their tolerances.
+
+The keep decisions are integers and are compared bit-exactly: with V an identity block the
+forward's O is P o M itself, and with dO an identity block the backward's dV is (P o M)ᵀ,
+so their zero patterns are the masks the kernels drew.  Values are compared within the
+forward / backward tolerances."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_111_b200 as fa
+import oracle.dropout as od
+from exact_attention_111_b200.inputs import random_blockmask, workloads, workload_inputs
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def _fwd(inp, causal, mask, p, seed):
+    q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
+    o, lse = fa.attention_forward(q, k, v, causal=causal, blockmask=P.to_dev(mask), dropout_p=p, dropout_seed=seed)
+    fa.fa_check_status()
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def _bwd(inp, o, lse, causal, mask, p, seed, deterministic=False):
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "dout"))
+    dq, dk, dv = fa.attention_backward(q, k, v, o, lse, do, causal=causal, blockmask=P.to_dev(mask),
+                                       dropout_p=p, dropout_seed=seed, deterministic=deterministic)
+    fa.fa_check_status()
+    torch.cuda.synchronize()
+    return {"dq": dq, "dk": dk, "dv": dv}
+
+
+@pytest.mark.parametrize("B,H,N", [(2, 2, 256), (1, 3, 384)])
+def test_forward_mask_is_bit_exact(B, H, N):
+    """V = identity on one 128-key tile (zero elsewhere): O[i, j] = (P o M)[i, 128 kt + j]."""
+    P.ensure_built()
+    p, seed = 0.3, 0x0123_4567_89AB_CDEF
+    base = P.inputs(B, H, N, 128, seed=6000 + N)
+    for kt in range(N // 128):
+        inp = dict(base)
+        v = torch.zeros((B, H, N, 128), dtype=torch.bfloat16)
+        v[:, :, 128 * kt:128 * (kt + 1)] = torch.eye(128, dtype=torch.bfloat16)
+        inp["v"] = v
+        o, _ = _fwd(inp, False, None, p, seed)
+        kept = (o.float() != 0).cpu().numpy()
+        for b in range(B):
+            for h in range(H):
+                ref = od.keep_mask(b * H + h, N, N, seed, p)[:, 128 * kt:128 * (kt + 1)]
+                assert np.array_equal(kept[b, h], ref), (b, h, kt)
+
+
+def test_backward_mask_is_bit_exact():
+    """dO = identity on query rows 0..127 (zero elsewhere): dV[j, c] = (P o M)[c, j]."""
+    P.ensure_built()
+    B, H, N, p, seed = 2, 2, 384, 0.45, 987654321
+    inp = P.inputs(B, H, N, 128, seed=6100)
+    o, lse = _fwd(inp, False, None, p, seed)
+    do = torch.zeros((B, H, N, 128), dtype=torch.bfloat16)
+    do[:, :, :128] = torch.eye(128, dtype=torch.bfloat16)
+    inp2 = dict(inp)
+    inp2["dout"] = do
+    g = _bwd(inp2, o, lse, False, None, p, seed)
+    kept = (g["dv"].float() != 0).cpu().numpy()         # [B, H, N keys, 128 query rows]
+    for b in range(B):
+        for h in range(H):
+            ref = od.keep_mask(b * H + h, N, N, seed, p)[:128, :].T
+            assert np.array_equal(kept[b, h], ref), (b, h)
+
+
+CASES = [
+    # B, H, N, d, causal, mask, p, dtype
+    (1, 2, 128, 64, False, False, 0.1, torch.bfloat16),
+    (2, 2, 300, 64, True, False, 0.5, torch.bfloat16),
+    (1, 2, 1000, 128, False, False, 0.2, torch.bfloat16),
+    (1, 2, 1000, 128, True, False, 0.1, torch.bfloat16),
+    (2, 1, 777, 64, False, True, 0.3, torch.bfloat16),
+    (1, 2, 640, 128, True, True, 0.9, torch.bfloat16),
+    (1, 2, 500, 64, True, False, 0.25, torch.float16),
+    (1, 1, 129, 128, False, False, 0.6, torch.float16),
+]
+
+
+def _oracle(inp, causal, mask, p, seed):
+    d = inp["q"].shape[-1]
+    return od.attention_bwd_dropout(inp["q"], inp["k"], inp["v"], inp["dout"], 1.0 / np.sqrt(d), p, seed, causal,
+                                    None if mask is None else mask.numpy())
+
+
+@pytest.mark.parametrize("B,H,N,d,causal,use_mask,p,dtype", CASES)
+def test_dropout_matches_oracle(B, H, N, d, causal, use_mask, p, dtype):
+    P.ensure_built()
+    seed = 1000 + N + d
+    inp = P.inputs(B, H, N, d, seed=6200 + N + d, dtype=dtype)
+    mask = None
+    if use_mask:
+        mask = random_blockmask((N + 127) // 128, 0.5, seed=4, keep_diagonal=False)
+        mask[0, :] = 0
+    o, lse = _fwd(inp, causal, mask, p, seed)
+    dq, dk, dv, o_ref, lse_ref = _oracle(inp, causal, mask, p, seed)
+    P.check_forward(o, lse, o_ref, lse_ref, o16_dtype=dtype, label=f"dropout p={p}", o_tol=P.O_TOL * od.keep_scale(p))
+    got = _bwd(inp, o, lse, causal, mask, p, seed)
+    P.check_grads(got, {"dq": dq, "dk": dk, "dv": dv}, label=f"dropout p={p}")
+
+
+def test_p_zero_is_the_plain_path_and_seeds_matter():
+    P.ensure_built()
+    inp = P.inputs(1, 2, 700, 64, seed=6300)
+    q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
+    o0, l0 = fa.attention_forward(q, k, v, causal=True)
+    o1, l1 = fa.attention_forward(q, k, v, causal=True, dropout_p=0.0, dropout_seed=5)
+    a1, _ = fa.attention_forward(q, k, v, causal=True, dropout_p=0.2, dropout_seed=5)
+    a2, _ = fa.attention_forward(q, k, v, causal=True, dropout_p=0.2, dropout_seed=5)
+    b1, lb = fa.attention_forward(q, k, v, causal=True, dropout_p=0.2, dropout_seed=6)
+    torch.cuda.synchronize()
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)
+    assert torch.equal(a1, a2)                       # same seed: same mask, same bits
+    assert not torch.equal(a1, b1)                   # another seed: another mask
+    assert torch.equal(lb, l0)                       # LSE is that of the undropped scores
+
+
+def test_dropout_with_deterministic_backward_repeats_bitwise():
+    P.ensure_built()
+    inp = P.inputs(2, 4, 2048, 64, seed=6400)
+    o, lse = _fwd(inp, False, None, 0.1, 77)
+    a = _bwd(inp, o, lse, False, None, 0.1, 77, deterministic=True)
+    b = _bwd(inp, o, lse, False, None, 0.1, 77, deterministic=True)
+    for n in ("dq", "dk", "dv"):
+        assert torch.equal(a[n], b[n]), n
+
+
+def test_dropout_full_size_sampled_heads():
+    P.ensure_built()
+    w = workloads()["gpt2_B64_H16_N1024_d64"]
+    inp = workload_inputs(w)
+    p, seed = 0.1, 2718281828
+    o, lse = _fwd(inp, False, None, p, seed)
+    got = _bwd(inp, o, lse, False, None, p, seed)
+    heads = P.sample_heads(w.B, w.H, 3, seed=6500)
+    dq, dk, dv, o_ref, lse_ref = od.attention_bwd_dropout(inp["q"], inp["k"], inp["v"], inp["dout"], w.scale, p,
+                                                          seed, heads=heads)
+    P.check_forward(o, lse, o_ref, lse_ref, heads=heads, o16_dtype=torch.bfloat16, label="dropout full size",
+                    o_tol=P.O_TOL * od.keep_scale(p))
+    P.check_grads(got, {"dq": dq, "dk": dk, "dv": dv}, heads=heads, label="dropout full size")
