@@ -453,6 +453,94 @@ def run_ours(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_fp8(args, w, world, rank, local):
+    """FP8 (E4M3) forward alone: one step = the V transpose + the fused forward over one batch
+    of the workload, quantized per tensor (there is no FP8 backward)."""
+    import torch
+    import exact_attention_111_b200 as fa
+    from exact_attention_111_b200.inputs import attention_flops, butterfly_blockmask, make_inputs, quantize_e4m3
+
+    fa.lib()
+    if w.d != 128:
+        raise SystemExit("--fp8 needs a d = 128 workload")
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    inp = make_inputs(w.B, w.H, w.N, w.d, rank_seed(w.seed, rank), k_scale=w.k_scale, with_dout=False)
+    qz = {n: quantize_e4m3(inp[n]) for n in ("q", "k", "v")}
+    host = {n: qz[n][0].view(torch.uint8).pin_memory() for n in qz}
+    d8 = {n: t.to(dev) for n, t in host.items()}
+    ds = {n: qz[n][1] for n in qz}
+    mask = butterfly_blockmask(w.tiles).to(dev) if w.butterfly else None
+    B, H, N, D = w.B, w.H, w.N, w.d
+    o = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    wsb = fa.fa_fwd_fp8_workspace_bytes(B, H, N, D)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(src):
+        fa.fa_fwd_fp8(src["q"], src["k"], src["v"], ds["q"], ds["k"], ds["v"], o, lse, B, H, N, D, w.scale, w.causal,
+                      mask, False, ws, wsb, stream)
+
+    for _ in range(args.warmup):
+        step(d8)
+    fa.fa_check_status(stream)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.25)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step(d8)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier(world)
+    fa.fa_check_status(stream)
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world)
+    flops = attention_flops(B, H, N, D, w.causal, False)
+    value = aggregate_tflops(world, flops, args.steps, elapsed_ms)
+    # end to end: E4M3 codes up from pinned host memory, O and LSE back, every step
+    host_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    host_l = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 20))
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    s0.record(stream)
+    for _ in range(e2e_steps):
+        for n in d8:
+            d8[n].copy_(host[n], non_blocking=True)
+        step(d8)
+        host_o.copy_(o, non_blocking=True)
+        host_l.copy_(lse, non_blocking=True)
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    peak8 = 2.0 * float(peaks["bf16_tflops"])
+    tf = value / world
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": dict(workload_config(w, world), mode="fp8 forward only (E4M3 Q, K, V with per-tensor "
+                                                      "dequantisation; V transpose + fused forward per step)"),
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": peak8, "unit": "TFLOP/s", "frac": tf / peak8,
+                     "traffic": None, "kernel": "fwd_fp8 (+ vt transpose)",
+                     "peak_source": f"2 x bf16_tflops of {peak_src} (MEASURED_PEAKS.json x nominal fp8/bf16 ratio)"},
+        "e2e": {"value": aggregate_tflops(world, flops, e2e_steps, e2e_ms), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sum(t.numel() for t in host.values()),
+                "d2h_bytes_per_step": host_o.numel() * 2 + host_l.numel() * 4, "steps": e2e_steps},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -467,6 +555,8 @@ def main():
                          "GPU; default: the workload's own setting)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="fused dropout probability in both passes (default 0: none)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the FP8 (E4M3) forward alone on the workload (d = 128)")
     ap.add_argument("--deterministic", action="store_true",
                     help="backward in deterministic mode (bitwise repeatable dQ)")
     args = ap.parse_args()
@@ -484,7 +574,7 @@ def main():
         return
     world, rank, local = dist_setup()
     try:
-        run_ours(args, w, world, rank, local)
+        (run_fp8 if args.fp8 else run_ours)(args, w, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

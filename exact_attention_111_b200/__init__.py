@@ -4,7 +4,7 @@ The binding marshals arguments only; every step of the computation runs in the C
 kernels behind the C ABI of ``include/fa.h``.  The C entry points are mirrored one to one
 (``fa_fwd``, ``fa_bwd``, ``fa_fwd_ex``, ``fa_bwd_ex``, ``fa_bwd_workspace_bytes``,
 ``fa_bwd_workspace_bytes_ex``, ``fa_bwd_noalloc``, ``fa_fwd_partial``, ``fa_lse_merge``, ``fa_fwd_splitkv``,
-``fa_fwd_splitkv_workspace_bytes``, ``fa_splitkv_choose``, ``fa_check_status``,
+``fa_fwd_splitkv_workspace_bytes``, ``fa_splitkv_choose``, ``fa_fwd_fp8``, ``fa_fwd_fp8_workspace_bytes``, ``fa_check_status``,
 ``fa_status_string``, ``fa_last_launch_count``); they take torch tensors (or raw device
 addresses as ints).  ``attention_forward`` / ``attention_backward`` /
 ``attention_forward_splitkv`` / ``attention_forward_partial`` / ``lse_merge`` and
@@ -24,7 +24,8 @@ __all__ = [
     "attention_forward", "attention_backward", "FlashAttention", "FA_BF16", "FA_FP16", "FA_FP32",
     "fa_fwd_partial", "fa_lse_merge", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes",
     "fa_splitkv_choose", "attention_forward_splitkv", "attention_forward_partial", "lse_merge",
-    "FA_MAX_PARTS", "fa_bwd_workspace_bytes_ex", "FA_ERR_RANGE",
+    "FA_MAX_PARTS", "fa_bwd_workspace_bytes_ex", "FA_ERR_RANGE", "fa_fwd_fp8", "fa_fwd_fp8_workspace_bytes",
+    "attention_forward_fp8",
 ]
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE, FA_ERR_RANGE = range(7)
@@ -65,6 +66,14 @@ class PartialArgs(ctypes.Structure):
     _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("o_part", _vp), ("lse_part", _vp),
                 ("B", _i), ("H", _i), ("N", _i), ("Nk", _i), ("d", _i), ("key_offset", _i),
                 ("scale", _f), ("causal", _i), ("blockmask", _vp), ("dtype", _i), ("stream", _vp)]
+
+
+class Fp8Args(ctypes.Structure):
+    """Mirror of fa_fwd_fp8_args."""
+    _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("descale_q", _f), ("descale_k", _f), ("descale_v", _f),
+                ("o", _vp), ("lse", _vp), ("B", _i), ("H", _i), ("N", _i), ("d", _i), ("scale", _f),
+                ("causal", _i), ("blockmask", _vp), ("o_fp32", _i), ("workspace", _vp),
+                ("workspace_bytes", ctypes.c_size_t), ("stream", _vp)]
 
 
 class FAError(RuntimeError):
@@ -111,6 +120,10 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
     L.fa_splitkv_choose.argtypes = [_i, _i, _i, _i, _i]
     L.fa_splitkv_choose.restype = _i
+    L.fa_fwd_fp8.argtypes = [ctypes.POINTER(Fp8Args)]
+    L.fa_fwd_fp8.restype = _i
+    L.fa_fwd_fp8_workspace_bytes.argtypes = [_i, _i, _i, _i]
+    L.fa_fwd_fp8_workspace_bytes.restype = ctypes.c_size_t
     _lib = L
     return L
 
@@ -220,6 +233,18 @@ def fa_fwd_splitkv(q, k, v, o, lse, B, H, N, d, scale, causal, blockmask, num_sp
                                 workspace_bytes, _stream(stream)), "fa_fwd_splitkv")
 
 
+def fa_fwd_fp8_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return lib().fa_fwd_fp8_workspace_bytes(B, H, N, d)
+
+
+def fa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, B, H, N, d, scale, causal=False,
+               blockmask=None, o_fp32=False, workspace=None, workspace_bytes=0, stream=None):
+    a = Fp8Args(_ptr(q8), _ptr(k8), _ptr(v8), float(descale_q), float(descale_k), float(descale_v), _ptr(o),
+                _ptr(lse), B, H, N, d, scale, int(bool(causal)), _ptr(blockmask), int(bool(o_fp32)),
+                _ptr(workspace), workspace_bytes, _stream(stream))
+    _check(lib().fa_fwd_fp8(ctypes.byref(a)), "fa_fwd_fp8")
+
+
 def _event(e):
     if e is None or isinstance(e, int):
         return e
@@ -321,6 +346,25 @@ def lse_merge(o_parts, lse_parts, out_dtype=None, stream=None):
     o = torch.empty((B, H, N, d), dtype=out_dtype, device=o_parts[0].device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=o_parts[0].device)
     fa_lse_merge(list(o_parts), list(lse_parts), o, lse, B, H, N, d, code, stream)
+    return o, lse
+
+
+def attention_forward_fp8(q8, k8, v8, descale_q, descale_k, descale_v, causal=False, blockmask=None, scale=None,
+                          o_fp32=False, workspace=None, stream=None):
+    """FP8 forward on E4M3 tensors [B, H, N, 128] (torch.float8_e4m3fn or uint8 codes) with
+    per-tensor dequantisation factors.  Returns (O bf16 or fp32, LSE)."""
+    import torch
+    for t in (q8, k8, v8):
+        if not (t.is_cuda and t.is_contiguous() and t.dim() == 4 and t.element_size() == 1):
+            raise ValueError("expected contiguous 8-bit CUDA tensors of shape [B, H, N, 128]")
+    B, H, N, d = q8.shape
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    o = torch.empty((B, H, N, d), dtype=torch.float32 if o_fp32 else torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    if workspace is None:
+        workspace = torch.empty(max(fa_fwd_fp8_workspace_bytes(B, H, N, d), 1), dtype=torch.uint8, device=q8.device)
+    fa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, B, H, N, d, scale, causal, blockmask, o_fp32,
+               workspace, workspace.numel(), stream)
     return o, lse
 
 

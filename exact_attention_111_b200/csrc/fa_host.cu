@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_fp8.h"
 #include "fa_internal.h"
 
 namespace fa {
@@ -64,6 +65,18 @@ bool encode_dqacc(CUtensorMap* m, const void* base, int BH, int N, int d) {
   const cuuint32_t box[3] = {32, 32, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 8-bit tensor with an innermost extent of 128-byte rows: 3-D map [z, y, x] with a
+// 128 x 128 x 1 box, 128-byte swizzle; elements past the extents read as zero.
+bool encode_u8(CUtensorMap* m, const void* base, int x, int y, int z) {
+  const cuuint64_t dims[3] = {(cuuint64_t)x, (cuuint64_t)y, (cuuint64_t)z};
+  const cuuint64_t strides[2] = {(cuuint64_t)x, (cuuint64_t)x * y};
+  const cuuint32_t box[3] = {128, (cuuint32_t)kTile, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -477,6 +490,57 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   m.n_parts = s_eff;
   m.out_kind = FA_BF16;
   if (launch_merge(m, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  t_last_launches = 2;
+  return FA_OK;
+}
+
+size_t fa_fwd_fp8_workspace_bytes(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, 1.f, FA_BF16) != FA_OK || d != 128) return 0;
+  const size_t Np = (size_t)((N + kTile - 1) / kTile) * kTile;
+  return align256((size_t)B * H * 128 * Np);
+}
+
+int fa_fwd_fp8(const fa_fwd_fp8_args* p) {
+  if (p == nullptr) return FA_ERR_INVALID_ARG;
+  const fa_fwd_fp8_args& x = *p;
+  int rc = check_shape(x.B, x.H, x.N, x.d, x.scale, FA_BF16);
+  if (rc != FA_OK) return rc;
+  if (x.d != 128) return FA_ERR_UNSUPPORTED;
+  for (float f : {x.descale_q, x.descale_k, x.descale_v})
+    if (!(f > 0.f) || !std::isfinite(f)) return FA_ERR_INVALID_ARG;
+  if (!x.q || !x.k || !x.v || !x.o || !x.lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(x.q, 16) || !aligned(x.k, 16) || !aligned(x.v, 16) || !aligned(x.o, 16) || !aligned(x.lse, 4))
+    return FA_ERR_INVALID_ARG;
+  const size_t need = fa_fwd_fp8_workspace_bytes(x.B, x.H, x.N, x.d);
+  if (!x.workspace || !aligned(x.workspace, 256) || x.workspace_bytes < need) return FA_ERR_WORKSPACE;
+  const int BH = x.B * x.H;
+  const int T = (x.N + kTile - 1) / kTile;
+  const int Np = T * kTile;
+  if (!fwd_grid_ok(BH, (T + 1) / 2, 1)) return FA_ERR_UNSUPPORTED;
+  if (!get_encode()) return FA_ERR_CUDA;
+  CUtensorMap tq, tk, tvt;
+  if (!encode_u8(&tq, x.q, 128, x.N, BH) || !encode_u8(&tk, x.k, 128, x.N, BH) ||
+      !encode_u8(&tvt, x.workspace, Np, 128, BH))
+    return FA_ERR_CUDA;
+  F8Args a{};
+  a.o = x.o;
+  a.lse = x.lse;
+  a.blockmask = x.blockmask;
+  if (status_word(&a.status) != FA_OK) return FA_ERR_CUDA;
+  a.timeout_ns = kWaitLimitNs;
+  a.N = x.N;
+  a.BH = BH;
+  a.T = T;
+  a.n_units = (T + 1) / 2;
+  a.group_heads = group_heads_for(BH, a.n_units);
+  a.causal = x.causal != 0;
+  a.o_fp32 = x.o_fp32 != 0;
+  a.scale_log2 = (float)((double)x.scale * x.descale_q * x.descale_k * 1.4426950408889634);
+  a.o_scale = x.descale_v / 256.0f;
+  t_last_launches = 0;
+  if (launch_fwd_fp8(tq, tk, tvt, a, static_cast<const uint8_t*>(x.v), static_cast<uint8_t*>(x.workspace), Np,
+                     static_cast<cudaStream_t>(x.stream)) != cudaSuccess)
+    return FA_ERR_CUDA;
   t_last_launches = 2;
   return FA_OK;
 }

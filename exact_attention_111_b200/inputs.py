@@ -119,3 +119,13 @@ def attention_flops(B: int, H: int, N: int, d: int, causal: bool, backward: bool
     if causal:
         f *= 0.5
     return f
+
+
+def quantize_e4m3(x: torch.Tensor):
+    """Per-tensor E4M3 codes of x: descale = max|x| / 448 and codes = E4M3(x / descale)
+    (round to nearest even, torch.float8_e4m3fn).  Returns (codes, descale); the values
+    the codes stand for are codes * descale."""
+    amax = float(x.float().abs().max())
+    descale = amax / 448.0 if amax > 0 else 1.0
+    codes = (x.float() / descale).to(torch.float8_e4m3fn)
+    return codes, descale

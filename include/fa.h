@@ -290,6 +290,44 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
  */
 int fa_splitkv_choose(int B, int H, int N, int causal, int num_sms);
 
+/*
+ * ---------------------------------------------------------------------------------------
+ * FP8 (E4M3) forward, head dimension 128.  The FlashAttention-2 wiki ("FlashAttention-3")
+ * names FP8 low precision for the Hopper follow-on without a scaling convention; here each
+ * of Q, K, V is given as E4M3 codes (OCP FP8 E4M3, the "fn" variant: finite, max 448) with
+ * one fp32 dequantisation factor per tensor, value = descale * code.
+ *
+ * The result is the exact attention of those values, O = softmax(scale * Q Kᵀ) V, up to one
+ * rounding: the probabilities enter the P V product as E4M3(256 P) / 256, i.e. with relative
+ * error <= 2^-4 (absolute <= 2^-18 below E4M3's normal range), so elementwise
+ *     |O - O_exact| <= 2^-4 * sum_j P_ij |V_jc| + 2^-18 * sum_j |V_jc|  (+ fp32 / output rounding).
+ * LSE is computed from the unrounded P in fp32, as in fa_fwd.
+ *   q, k, v   : in,  E4M3 bytes [B, H, N, 128], 16-byte aligned
+ *   o         : out, [B, H, N, 128] bf16, or fp32 when o_fp32 != 0
+ *   lse       : out, [B, H, N] fp32
+ *   workspace : device scratch of fa_fwd_fp8_workspace_bytes(B, H, N, 128) bytes, 256-byte
+ *               aligned: V transposed to [B, H, 128, ceil(N/128)*128] (keys contiguous)
+ * causal and blockmask as for fa_fwd.  Two launches (the V transpose, then the fused
+ * forward).  d != 128 returns FA_ERR_UNSUPPORTED; a descale that is not finite and > 0
+ * returns FA_ERR_INVALID_ARG.  There is no FP8 backward.
+ */
+typedef struct {
+  const void* q; const void* k; const void* v;
+  float descale_q, descale_k, descale_v;
+  void* o;
+  float* lse;
+  int B, H, N, d;
+  float scale;
+  int causal;
+  const uint8_t* blockmask;
+  int o_fp32;
+  void* workspace; size_t workspace_bytes;
+  void* stream;
+} fa_fwd_fp8_args;
+
+size_t fa_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
+int fa_fwd_fp8(const fa_fwd_fp8_args* args);
+
 /* Static human-readable name of a status code. */
 const char* fa_status_string(int status);
 

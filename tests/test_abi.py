@@ -259,3 +259,27 @@ def test_dropout_argument_errors(L):
         b = fa.BwdArgs(*([FAKE] * 9), 1, 1, 128, 64, 0.125, 0, None, fa.FA_BF16, None, 0x100000, ws, None, None, None,
                        0, p, 1)
         assert L.fa_bwd_ex(ct.byref(b)) == fa.FA_ERR_INVALID_ARG, p
+
+
+def test_fp8_workspace_and_argument_errors(L):
+    import ctypes as ct
+    for B, H, N in ((1, 1, 128), (2, 3, 1000), (1, 1, 1)):
+        Np = (N + 127) // 128 * 128
+        assert fa.fa_fwd_fp8_workspace_bytes(B, H, N, 128) == (B * H * 128 * Np + 255) // 256 * 256
+    assert fa.fa_fwd_fp8_workspace_bytes(1, 1, 128, 64) == 0
+    ws = fa.fa_fwd_fp8_workspace_bytes(1, 1, 256, 128)
+
+    def call(**kw):
+        a = dict(d=128, dq=0.5, dk=0.5, dv=0.5, q=FAKE, ws=0x100000, wsb=ws, N=256)
+        a.update(kw)
+        args = fa.Fp8Args(a["q"], FAKE, FAKE, a["dq"], a["dk"], a["dv"], FAKE, FAKE, 1, 1, a["N"], a["d"], 0.088,
+                          0, None, 0, a["ws"], a["wsb"], None)
+        return L.fa_fwd_fp8(ct.byref(args))
+    assert call(d=64) == fa.FA_ERR_UNSUPPORTED
+    assert call(dq=0.0) == fa.FA_ERR_INVALID_ARG
+    assert call(dv=float("inf")) == fa.FA_ERR_INVALID_ARG
+    assert call(dk=float("nan")) == fa.FA_ERR_INVALID_ARG
+    assert call(q=FAKE + 8) == fa.FA_ERR_INVALID_ARG
+    assert call(wsb=ws - 1) == fa.FA_ERR_WORKSPACE
+    assert call(ws=0x100000 + 128) == fa.FA_ERR_WORKSPACE
+    assert L.fa_fwd_fp8(None) == fa.FA_ERR_INVALID_ARG
