@@ -46,6 +46,10 @@ constexpr int kF8SmemTiles = 2 * kF8TileBytes           // Q (two query tiles)
                              + 2 * kF8Stages * kF8TileBytes  // K and Vᵀ rings
                              + 2 * kF8TileBytes;          // P (two query tiles)
 constexpr float kF8PScale = 256.0f;
+// exp2 pairs per 8 evaluated by the FMA-pipe polynomial instead of the SFU: the SFU is this
+// kernel's tightest pipe once the products run at the 8-bit rate (measured at N = 4096 and
+// 16384: 2 of 8 is 7 % faster than none; 4 of 8 is slower than none)
+constexpr int kF8PolyOf8 = 2;
 constexpr float kLn2F8 = 0.693147180559945309f;
 
 struct F8Shared {
@@ -337,7 +341,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float2 t = fma2(make_float2(s[32 * h + 2 * i], s[32 * h + 2 * i + 1]), sl2v, mnegv);
-          const float2 p = make_float2(ex2(t.x), ex2(t.y));
+          const float2 p = (((16 * h + i) & 7) < kF8PolyOf8) ? exp2_poly2(t) : make_float2(ex2(t.x), ex2(t.y));
           acc[i & 3] = add2(acc[i & 3], p);
           const float2 ps = mul2(p, p256);
           const uint32_t b2 = pack_e4m3x2(ps.x, ps.y);
