@@ -26,7 +26,7 @@ calculus -- the pages name backward recomputation but print no formula):
     dV = Pᵀ dO,   dP = dO Vᵀ,   D_i = sum_j P_ij dP_ij,
     dS = P o (dP - D),   dQ = scale * dS K,   dK = scale * dSᵀ Q
 
-Readings of points the pages leave open (each listed in the design doc):
+Readings of points the pages leave open:
   * scale: the pages write softmax(QKᵀ)V with no scale; a caller-supplied ``scale``
     multiplies QKᵀ (1/sqrt(d) in every workload).
   * causal: key j is visible to query i iff j <= i (top-left aligned, equal lengths).

@@ -6,7 +6,7 @@ CPU legs may import it, and it shares no code with the CUDA path.
 The pages fuse dropout into the attention kernel and regenerate its mask in the backward
 pass from the saved random-generator state instead of storing it (FlashAttention-NeurIPS22
 summary, "核心方法 / Kernel fusion" and "Backward recomputation").  They fix neither the
-generator nor the mask layout; the readings taken here (each listed in the design doc):
+generator nor the mask layout; the readings taken here:
 
   * generator: Philox4x32-10, the counter-based generator of Salmon, Moraes, Dror and
     Shaw, "Parallel random numbers: as easy as 1, 2, 3" (SC'11): a 128-bit counter and a
