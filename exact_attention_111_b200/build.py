@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfa.so")
-SOURCES = ["fa_host.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_merge.cu", "fa_fwd_fp8.cu", "fa_noalloc.cu"]
+SOURCES = ["fa_host.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_merge.cu", "fa_fwd_fp8.cu", "fa_selftest.cu", "fa_noalloc.cu"]
 HEADERS = ["fa_internal.h", "sm100.cuh", "fa_fp8.h"]
 
 

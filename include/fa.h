@@ -328,6 +328,18 @@ typedef struct {
 size_t fa_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
 int fa_fwd_fp8(const fa_fwd_fp8_args* args);
 
+/*
+ * Diagnostic of failure detection (no counterpart in the pages).  Launches one small kernel
+ * that runs the library's bounded mbarrier wait on a barrier nothing ever completes, with
+ * a limit of limit_us microseconds (1 .. 1000000).  The wait must give up at the limit and
+ * the kernel return; the next fa_check_status on `stream` then returns FA_ERR_TIMEOUT (and
+ * clears the word).  waited_ok: NULL, or a device int that receives 0 when the wait gave up
+ * (1 would mean the barrier completed, which cannot happen).  Nothing faults, traps or
+ * loops without bound.  Returns FA_OK once launched, FA_ERR_INVALID_ARG for a limit out of
+ * range, FA_ERR_CUDA on a launch error.
+ */
+int fa_selftest_wait_timeout(unsigned int limit_us, int* waited_ok, void* stream);
+
 /* Static human-readable name of a status code. */
 const char* fa_status_string(int status);
 

@@ -283,3 +283,8 @@ def test_fp8_workspace_and_argument_errors(L):
     assert call(wsb=ws - 1) == fa.FA_ERR_WORKSPACE
     assert call(ws=0x100000 + 128) == fa.FA_ERR_WORKSPACE
     assert L.fa_fwd_fp8(None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_selftest_argument_errors(L):
+    assert L.fa_selftest_wait_timeout(0, None, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_selftest_wait_timeout(1000001, None, None) == fa.FA_ERR_INVALID_ARG
