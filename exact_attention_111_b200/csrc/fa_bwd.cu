@@ -29,7 +29,9 @@
 //
 // bwd_main roles (320 threads): warps 0-7 two compute groups, one key row per thread (TMEM
 // lanes), each group owning half of the query columns and draining half of each dQ partial;
-// warp 8 TMA producer; warp 9 MMA issuer.
+// warp 8 TMA producer; warp 9 MMA issuer.  At d = 64 in the default mode, four groups (warps
+// 0-15, a quarter of the query columns each; groups 0 and 1 also drain dQ and write dV / dK),
+// producer warp 16, MMA warp 17.
 // Tensor memory: Sᵀ/Pᵀ [0,128) (Pᵀ as 16-bit over columns [0,32) and [64,96)), dPᵀ [128,256),
 // dV and dK after them; dQ shares the dPᵀ columns when d = 128 and has its own for d = 64.
 // Per query tile, the MMAs: Sᵀ = K Q_iᵀ, dPᵀ = V dO_iᵀ, dV += Pᵀ dO_i (Pᵀ from TMEM),
@@ -171,8 +173,10 @@ struct BwdCfg {
 };
 
 constexpr int kBwdThreads = 320;   // 2 compute groups (8 warps), producer, MMA issuer
-constexpr int kBwdLoadWarp = 8;
-constexpr int kBwdMmaWarp = 9;
+// d = 64, default mode: four compute groups of 32 query columns (18 warps, 96 registers) instead
+// of two.  The twice as many warps hide the phase latencies that bound this kernel at d = 64
+// (measured backward main: +5 to +7 % from N = 512 to 16384, causal included).
+constexpr bool kBwdFourGroups = true;
 
 struct BwdBars {
   uint64_t kv_full;
@@ -242,12 +246,18 @@ __device__ __forceinline__ int next_kept(int k, int j, int T, int causal, const 
   return k;
 }
 
-template <int D, bool kFp16, bool kDet, bool kDrop>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+// kG compute groups of 128 threads, each owning 128 / kG query columns of every tile: kG = 2
+// (the default) or kG = 4 (d = 64, default mode: twice the warps to hide phase latencies; the
+// dQ drain and the dV / dK epilogue stay with groups 0 and 1).
+template <int D, bool kFp16, bool kDet, bool kDrop, int kG>
+__global__ void __launch_bounds__(128 * kG + 64, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
   using C = BwdCfg<D>;
+  static_assert(kG == 2 || (kG == 4 && D == 64 && !kDet && !kDrop), "four groups: d = 64, default mode");
+  constexpr int kLoadW = 4 * kG, kMmaW = 4 * kG + 1;
+  constexpr int kCols = kTile / kG;                 // query columns per compute group
   extern __shared__ __align__(1024) uint8_t smem[];
   BwdBars& sh = *reinterpret_cast<BwdBars*>(smem + C::oBAR);
   const int warp = warp_id(), lane = lane_id();
@@ -268,8 +278,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(&sh.s_full, 1);
     mbar_init(&sh.dp_full, 1);
-    mbar_init(&sh.p_full, 256);
-    mbar_init(&sh.ds_full, 256);
+    mbar_init(&sh.p_full, 128 * kG);
+    mbar_init(&sh.ds_full, 128 * kG);
     mbar_init(&sh.dq_full, 1);
     mbar_init(&sh.dq_empty, 256);
     mbar_init(&sh.mma_done, 1);
@@ -277,7 +287,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (!aligned) atomicCAS(a.status, 0, kDevBadState);
     fence_barrier_init();
   }
-  if (warp == kBwdMmaWarp) {
+  if (warp == kMmaW) {
     tmem_alloc(&sh.tmem_base, 512);
     tmem_relinquish();
   }
@@ -288,7 +298,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int k_first = next_kept(0, j, a.T, a.causal, a.blockmask);
   const bool any = aligned && k_first < a.T;
 
-  if (warp == kBwdLoadWarp) {
+  if (warp == kLoadW) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && any) {
       prefetch_tmap(&tm_q);
@@ -322,7 +332,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == kBwdMmaWarp) {
+  } else if (warp == kMmaW) {
     // ------------------------------------------------------------------ MMA issuer
     // Issue order per kept query tile c (stage s = c % 2):
     //   [Sᵀ(c), dPᵀ(c) issued one step earlier]  dV += Pᵀ(c) dO(c);  Sᵀ(c+1);
@@ -373,10 +383,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // dV += Pᵀ dO(c)   (Pᵀ read from tensor memory)
           if (!(ok = mbar_wait(&sh.p_full, c & 1, abort_flag, st))) break;
           tc_fence_after();
-          // Pᵀ query columns 16kk..16kk+15 sit in TMEM columns 64*(kk/4) + 8*(kk%4) (see the compute groups)
+          // Pᵀ query columns 16kk..16kk+15 sit in TMEM columns kCols*(16kk/kCols) + (16kk mod kCols)/2
+          // (each group packs its columns over the first half of its own Sᵀ range)
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + C::tDV, tmem + C::tS + (kk >> 2) * 64 + (kk & 3) * 8,
+            mma_ts(tmem + C::tDV, tmem + C::tS + (16 * kk / kCols) * kCols + ((16 * kk) % kCols) / 2,
                    smem_desc_sw128(dob + kk * 2048, C::kPanelBytes, 1024), id_kn, (c > 0 || kk > 0) ? 1u : 0u);
           // Sᵀ(c+1)
           if (more) {
@@ -438,7 +449,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tQ = tmem + C::tDQ + lane_off + kHalfD * g;
     const float sl2 = a.scale_log2;
     const bool key_ok = key < a.N;
-    uint8_t* ds_row = smem + C::oDS + g * C::kPanelBytes + r * 128;
+    // this group's columns of the key row's dSᵀ: panel (kCols g) / 64, first 16-byte chunk ds_c0
+    uint8_t* ds_row = smem + C::oDS + (kCols * g / 64) * C::kPanelBytes + r * 128;
+    constexpr int kChunks = kCols / 8;
+    const int ds_c0 = ((kCols * g) % 64) / 8;
     int c = 0;
     bool ok = true;
     int i_prev = -1;
@@ -529,25 +543,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
         tc_fence_after();
         // -LSE*log2(e) and -D of this group's 64 query columns (bulk-loaded with the stage)
-        const float* nlse2 = reinterpret_cast<const float*>(smem + C::oLSE + s * kTile * 4) + 64 * g;
-        const float* ndlt = reinterpret_cast<const float*>(smem + C::oDELTA + s * kTile * 4) + 64 * g;
+        const float* nlse2 = reinterpret_cast<const float*>(smem + C::oLSE + s * kTile * 4) + kCols * g;
+        const float* ndlt = reinterpret_cast<const float*>(smem + C::oDELTA + s * kTile * 4) + kCols * g;
         const bool diag = a.causal && (i == j);     // key r visible to query column q iff r <= q
         // Phase A: Pᵀ = 2^(scale*log2e*Sᵀ - LSE*log2e), 16-bit, over Sᵀ in TMEM.  Both
         // 32-column chunks are loaded before one wait; -LSE*log2e comes in float4s; the
         // exponent argument is one packed fp32 FMA per pair.
-        uint32_t pk[32];
+        uint32_t pk[kCols / 2];
         {
-          uint32_t sv[64];
-          tmem_ld32(tS + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          tmem_ld32(tS + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          uint32_t sv[kCols];
+#pragma unroll
+          for (int m = 0; m < kCols / 32; ++m) tmem_ld32(tS + kCols * g + 32 * m, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * m]));
           tmem_wait_ld();
-          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+#pragma unroll
+          for (int m = 0; m < kCols / 32; ++m) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sv[32 * m]));
           const float4* nl4 = reinterpret_cast<const float4*>(nlse2);
           const float2 sl2v = make_float2(sl2, sl2);
           const bool any_mask = !key_ok || diag;
 #pragma unroll
-          for (int t4 = 0; t4 < 16; ++t4) {            // 4 query columns per step
+          for (int t4 = 0; t4 < kCols / 4; ++t4) {     // 4 query columns per step
             const float4 nl = nl4[t4];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -556,7 +570,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                     hh == 0 ? make_float2(nl.x, nl.y) : make_float2(nl.z, nl.w));
               float2 p = ((t & 7) < C::kPolyOf8) ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
               if (any_mask) {
-                const int q0 = 64 * g + 2 * t;          // column within the tile
+                const int q0 = kCols * g + 2 * t;       // column within the tile
                 if (!key_ok || (diag && r > q0)) p.x = 0.f;
                 if (!key_ok || (diag && r > q0 + 1)) p.y = 0.f;
               }
@@ -582,13 +596,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tmem_st16(tS + 64 * g + 16 * h2, pd);
           }
         } else {
-          tmem_st32(tS + 64 * g, pk);
+          if constexpr (kCols == 64) tmem_st32(tS + 64 * g, pk);
+          else tmem_st16(tS + kCols * g, pk);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sh.p_full);
         // dQ of the previous query tile (its completion also frees the dSᵀ buffer)
-        if (c > 0) {
+        if (g < 2 && c > 0) {                       // groups 0 and 1 drain dQ
           ok = drain(i_prev, c - 1);
           if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
         }
@@ -597,16 +612,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
         tc_fence_after();
         {
-          uint32_t dpv[64];
-          tmem_ld32(tDP + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&dpv[0]));
-          tmem_ld32(tDP + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&dpv[32]));
-          tmem_wait_ld();
-          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dpv[0]));
-          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dpv[32]));
-          const float4* nd4 = reinterpret_cast<const float4*>(ndlt);
-          uint32_t w[32];
+          uint32_t dpv[kCols];
 #pragma unroll
-          for (int t4 = 0; t4 < 16; ++t4) {
+          for (int m = 0; m < kCols / 32; ++m) tmem_ld32(tDP + kCols * g + 32 * m, *reinterpret_cast<uint32_t(*)[32]>(&dpv[32 * m]));
+          tmem_wait_ld();
+#pragma unroll
+          for (int m = 0; m < kCols / 32; ++m) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dpv[32 * m]));
+          const float4* nd4 = reinterpret_cast<const float4*>(ndlt);
+          uint32_t w[kCols / 2];
+#pragma unroll
+          for (int t4 = 0; t4 < kCols / 4; ++t4) {
             const float4 nd = nd4[t4];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -626,8 +641,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!C::kOwnStaging) wait_stage_read();
           // 128 bytes = eight 16-byte chunks of this key row (128-byte swizzle)
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int chunk = t ^ (r & 7);
+          for (int t = 0; t < kChunks; ++t) {
+            const int chunk = (ds_c0 + t) ^ (r & 7);
             *reinterpret_cast<uint4*>(ds_row + chunk * 16) = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
           }
         }
@@ -636,13 +651,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive(&sh.ds_full);
         i_prev = i;
       }
-      if (ok && c > 0) ok = drain(i_prev, c - 1);
+      if (g < 2 && ok && c > 0) ok = drain(i_prev, c - 1);
       if (lane == 0) bulk_wait_all();
     }
     // Epilogue: group 0 writes dV, group 1 writes scale * dK, one key row per thread.
     if (ok) ok = mbar_wait(&sh.mma_done, 0, abort_flag, st);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    if (ok && g < 2) {
       tc_fence_after();
       const size_t base = ((size_t)bh * a.N + key) * D;
       const uint32_t tA = tmem + (g == 0 ? C::tDV : C::tDK) + lane_off;
@@ -675,7 +690,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kBwdMmaWarp) {
+  if (warp == kMmaW) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -686,12 +701,19 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t s) {
   using C = BwdCfg<D>;
   const bool drop = a.drop.t > 0;
-  auto kern = a.dq_fix != nullptr ? (drop ? bwd_kernel<D, kFp16, true, true> : bwd_kernel<D, kFp16, true, false>)
-                                  : (drop ? bwd_kernel<D, kFp16, false, true> : bwd_kernel<D, kFp16, false, false>);
+  auto kern = a.dq_fix != nullptr ? (drop ? bwd_kernel<D, kFp16, true, true, 2> : bwd_kernel<D, kFp16, true, false, 2>)
+                                  : (drop ? bwd_kernel<D, kFp16, false, true, 2> : bwd_kernel<D, kFp16, false, false, 2>);
+  int threads = kBwdThreads;
+  if constexpr (D == 64) {
+    if (kBwdFourGroups && a.dq_fix == nullptr && !drop) {
+      kern = bwd_kernel<D, kFp16, false, false, 4>;
+      threads = 4 * 128 + 64;
+    }
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.T);
-  kern<<<grid, kBwdThreads, C::kSmem, s>>>(tq, tk, tv, tdo, tdq, a);
+  kern<<<grid, threads, C::kSmem, s>>>(tq, tk, tv, tdo, tdq, a);
   return cudaGetLastError();
 }
 
