@@ -434,11 +434,11 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ key-row compute groups
-    // Group g (warps 4g..4g+3) owns query columns [64g, 64g+64) of every Sᵀ / dPᵀ tile; each
-    // thread owns one key row (TMEM lane).  P stays in registers between the two phases.
-    // The groups also drain each dQ partial (query rows on TMEM lanes, half the columns each)
-    // right after the next P phase: the columns are released as soon as they are read, and
-    // the fp32 atomics follow from registers.
+    // Group g (warps 4g..4g+3) owns query columns [kCols g, kCols (g+1)) of every Sᵀ / dPᵀ
+    // tile; each thread owns one key row (TMEM lane).  P stays in registers between the two
+    // phases.  Groups 0 and 1 also drain each dQ partial (query rows on TMEM lanes, half the
+    // columns each) right after the next P phase: the columns are released as soon as they
+    // are read, and the reduction into the accumulator follows from shared memory.
     const int g = warp >> 2;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;                   // key row within the tile == TMEM lane

@@ -13,6 +13,8 @@
 //   warp  8    TMA producer: Q once, then the K/V ring (no multicast)
 //   warp  9    MMA issuer (one elected thread) and TMEM allocator
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 [256+d, 256+2d).
+// (The one-query-tile layout of FwdCfg<D, 1>, used for short d = 64 sequences: softmax warps
+// 0-3, producer warp 4, MMA warp 5, 256 columns with S [0,128) and O [128,128+d).)
 // P (16-bit) is written over the first 64 columns of its S tile and consumed from TMEM by
 // the PV MMA.  Per key tile u the MMA thread issues, for each query tile q that keeps u:
 //   O_q += P_q(prev) V(prev)   then   S_q = Q_q K(u)ᵀ   (commit -> s_full[q]),
