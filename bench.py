@@ -13,6 +13,10 @@ Multi-GPU (torchrun, one process per GPU): heads are independent, so each rank r
 own batch of the workload with no data-path collective (weak scaling); the only
 communication is the barrier and the max-over-ranks of the device time.
 
+Modes (same JSON line, mode named in ``config``): ``--deterministic`` (int64 fixed-point dQ
+accumulation), ``--dropout P`` (fused dropout in both passes), ``--fwd-splits S`` (split-KV
+forward), ``--fp8`` (the FP8 E4M3 forward alone, d = 128).
+
 Prints one JSON line on rank 0.  ``--impl reference`` times the fp64 CPU oracle (the only
 other implementation of this computation available here) on a bounded sample of the same
 workload, on the host cores.
