@@ -4,7 +4,7 @@ The binding marshals arguments only; every step of the computation runs in the C
 kernels behind the C ABI of ``include/fa.h``.  The C entry points are mirrored one to one
 (``fa_fwd``, ``fa_bwd``, ``fa_fwd_ex``, ``fa_bwd_ex``, ``fa_bwd_workspace_bytes``,
 ``fa_bwd_workspace_bytes_ex``, ``fa_bwd_noalloc``, ``fa_fwd_partial``, ``fa_lse_merge``, ``fa_fwd_splitkv``,
-``fa_fwd_splitkv_workspace_bytes``, ``fa_splitkv_choose``, ``fa_fwd_fp8``, ``fa_fwd_fp8_workspace_bytes``, ``fa_selftest_wait_timeout``, ``fa_check_status``,
+``fa_fwd_splitkv_workspace_bytes``, ``fa_splitkv_choose``, ``fa_fwd_fp8``, ``fa_fwd_fp8_workspace_bytes``, ``fa_selftest_wait_timeout``, ``fa_selftest_exp2_poly``, ``fa_check_status``,
 ``fa_status_string``, ``fa_last_launch_count``); they take torch tensors (or raw device
 addresses as ints).  ``attention_forward`` / ``attention_backward`` /
 ``attention_forward_splitkv`` / ``attention_forward_partial`` / ``lse_merge`` and
@@ -25,7 +25,7 @@ __all__ = [
     "fa_fwd_partial", "fa_lse_merge", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes",
     "fa_splitkv_choose", "attention_forward_splitkv", "attention_forward_partial", "lse_merge",
     "FA_MAX_PARTS", "fa_bwd_workspace_bytes_ex", "FA_ERR_RANGE", "fa_fwd_fp8", "fa_fwd_fp8_workspace_bytes",
-    "attention_forward_fp8", "fa_selftest_wait_timeout",
+    "attention_forward_fp8", "fa_selftest_wait_timeout", "fa_selftest_exp2_poly",
 ]
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE, FA_ERR_RANGE = range(7)
@@ -126,6 +126,8 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_fp8_workspace_bytes.restype = ctypes.c_size_t
     L.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp, _vp]
     L.fa_selftest_wait_timeout.restype = _i
+    L.fa_selftest_exp2_poly.argtypes = [_vp, _vp, _i, _vp]
+    L.fa_selftest_exp2_poly.restype = _i
     _lib = L
     return L
 
@@ -239,6 +241,11 @@ def fa_selftest_wait_timeout(limit_us: int, waited_ok=None, stream=None):
     """Runs the bounded-wait diagnostic (include/fa.h); fa_check_status then reports
     FA_ERR_TIMEOUT."""
     _check(lib().fa_selftest_wait_timeout(int(limit_us), _ptr(waited_ok), _stream(stream)), "fa_selftest_wait_timeout")
+
+
+def fa_selftest_exp2_poly(x, y, n: int, stream=None):
+    """y[:n] = 2^x[:n] by the kernels' FMA-pipe polynomial (the diagnostic of include/fa.h)."""
+    _check(lib().fa_selftest_exp2_poly(_ptr(x), _ptr(y), int(n), _stream(stream)), "fa_selftest_exp2_poly")
 
 
 def fa_fwd_fp8_workspace_bytes(B: int, H: int, N: int, d: int) -> int:

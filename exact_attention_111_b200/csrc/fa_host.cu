@@ -178,6 +178,39 @@ int status_word(int** out) {
 
 }  // namespace
 
+// Public status for a nonzero device status word: a bounded wait that expired is
+// FA_ERR_TIMEOUT, a deterministic-backward partial out of range is FA_ERR_RANGE, and anything
+// else (kDevBadState: the kernel found its dynamic shared memory misaligned and did no work)
+// is FA_ERR_CUDA.
+int status_from_device_word(int v) {
+  switch (v) {
+    case kDevOk: return FA_OK;
+    case kDevTimeout: return FA_ERR_TIMEOUT;
+    case kDevRange: return FA_ERR_RANGE;
+    default: return FA_ERR_CUDA;
+  }
+}
+
+// Every check of a backward call that needs no CUDA call: shape, pointers, alignment, the
+// dropout probability and (check_workspace) the workspace.  Used by fa_bwd_ex and, before it
+// touches the device at all, by fa_bwd_noalloc.
+int validate_bwd(const fa_bwd_args& x, bool check_workspace) {
+  int rc = check_shape(x.B, x.H, x.N, x.d, x.scale, x.dtype);
+  if (rc != FA_OK) return rc;
+  if (!x.q || !x.k || !x.v || !x.o || !x.lse || !x.dout || !x.dq || !x.dk || !x.dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(x.q, 16) || !aligned(x.k, 16) || !aligned(x.v, 16) || !aligned(x.o, 16) || !aligned(x.dout, 16) ||
+      !aligned(x.dq, 16) || !aligned(x.dk, 16) || !aligned(x.dv, 16) || !aligned(x.lse, 4) ||
+      !aligned(x.visit_log, 4))
+    return FA_ERR_INVALID_ARG;
+  Dropout drop{};
+  if (!make_dropout(x.dropout_p, x.dropout_seed, &drop)) return FA_ERR_INVALID_ARG;
+  if (check_workspace) {
+    const WsLayout w = ws_layout(x.B, x.H, x.N, x.d, x.deterministic != 0);
+    if (!x.workspace || !aligned(x.workspace, 256) || x.workspace_bytes < w.total) return FA_ERR_WORKSPACE;
+  }
+  return FA_OK;
+}
+
 int* device_status_word() {
   int* p = nullptr;
   return status_word(&p) == FA_OK ? p : nullptr;
@@ -265,18 +298,12 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 int fa_bwd_ex(const fa_bwd_args* p) {
   if (p == nullptr) return FA_ERR_INVALID_ARG;
   const fa_bwd_args& x = *p;
-  int rc = check_shape(x.B, x.H, x.N, x.d, x.scale, x.dtype);
+  int rc = validate_bwd(x, true);
   if (rc != FA_OK) return rc;
-  if (!x.q || !x.k || !x.v || !x.o || !x.lse || !x.dout || !x.dq || !x.dk || !x.dv) return FA_ERR_INVALID_ARG;
-  if (!aligned(x.q, 16) || !aligned(x.k, 16) || !aligned(x.v, 16) || !aligned(x.o, 16) || !aligned(x.dout, 16) ||
-      !aligned(x.dq, 16) || !aligned(x.dk, 16) || !aligned(x.dv, 16) || !aligned(x.lse, 4) ||
-      !aligned(x.visit_log, 4))
-    return FA_ERR_INVALID_ARG;
   Dropout drop{};
-  if (!make_dropout(x.dropout_p, x.dropout_seed, &drop)) return FA_ERR_INVALID_ARG;
+  make_dropout(x.dropout_p, x.dropout_seed, &drop);
   const bool det = x.deterministic != 0;
   const WsLayout w = ws_layout(x.B, x.H, x.N, x.d, det);
-  if (!x.workspace || !aligned(x.workspace, 256) || x.workspace_bytes < w.total) return FA_ERR_WORKSPACE;
   const bool fp16 = x.dtype == FA_FP16;
   const int BH = x.B * x.H;
   const int T = (x.N + kTile - 1) / kTile;
@@ -554,7 +581,7 @@ int fa_check_status(void* stream) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
-    return v == kDevTimeout ? FA_ERR_TIMEOUT : v == kDevRange ? FA_ERR_RANGE : FA_ERR_CUDA;
+    return status_from_device_word(v);
   }
   return FA_OK;
 }

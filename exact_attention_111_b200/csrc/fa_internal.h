@@ -11,8 +11,10 @@ namespace fa {
 constexpr int kTile = 128;          // rows per query tile and keys per key/value tile
 constexpr int kMaxTiles = 2048;     // tile lists live in shared memory (N <= 2048 * 128)
 
-// Error codes a kernel can record in the device status word (read by fa_check_status).
-enum : int { kDevOk = 0, kDevTimeout = 4, kDevBadState = 6, kDevRange = 7 };
+// Error codes a kernel can record in the device status word.  They live in their own range
+// (0x100 and up), disjoint from the public fa_status values, and fa_check_status translates
+// each one explicitly (status_from_device_word): a device word is never returned as it is.
+enum : int { kDevOk = 0, kDevTimeout = 0x101, kDevBadState = 0x102, kDevRange = 0x103 };
 
 // Deterministic backward: dQ partials are added as int64 fixed point with 32 fraction bits.
 // Integer addition is associative, so the sum does not depend on the order in which the
@@ -124,6 +126,7 @@ cudaError_t launch_bwd_post(const BwdPostArgs& a, bool fp16, cudaStream_t s);
 cudaError_t launch_merge(const MergeArgs& a, int d, cudaStream_t s);
 
 int* device_status_word();  // address of the per-process device status word
+int status_from_device_word(int v);   // fa_status for a device status word
 
 // Heads per CTA-ordering group: about two waves of CTAs (148 SMs, one CTA each) per group, so
 // the heads a wave works on keep their tiles in L2 while each group still runs its heaviest

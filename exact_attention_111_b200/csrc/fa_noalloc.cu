@@ -9,7 +9,10 @@
 // file-scope device array instead, and the entry point allocates nothing.
 //
 // The array (kNoAllocScratchBytes) exists on every GPU that loads the library, until the
-// process exits.  Every call on a device shares that device's array, so calls that overlap
+// process exits.  The CUDA runtime loads device code lazily, so on each device the array's
+// memory is committed when this file's code is first loaded there -- by the first call's
+// address lookup -- and that first call must therefore come at start-up, before any stream
+// capture or freezing of the device memory pool.  Later calls allocate nothing.  Every call on a device shares that device's array, so calls that overlap
 // on the GPU (other streams, other host threads) race on it and must be serialised by the
 // caller.  The array keeps the last call's contents; the backward's first kernel rewrites
 // every part the later kernels read (it zeroes the dQ accumulator and writes both per-row
@@ -47,18 +50,26 @@ int scratch_for_current_device(void** out) {
 
 }  // namespace
 
+namespace fa {
+int validate_bwd(const fa_bwd_args& x, bool check_workspace);   // fa_host.cu
+}
+
 extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                               const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                               float scale, int causal, const uint8_t* blockmask, void* stream) {
-  const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
-  if (need == 0) {
-    // invalid shape: let the regular entry point report the precise argument error
-    return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockmask, nullptr, 0, stream);
-  }
-  if (need > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
-  void* scratch = nullptr;
-  const int rc = scratch_for_current_device(&scratch);
+  fa_bwd_args a{};
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.B = B; a.H = H; a.N = N; a.d = d; a.scale = scale; a.causal = causal; a.blockmask = blockmask;
+  a.dtype = FA_BF16; a.visit_log = nullptr; a.stream = stream;
+  // Argument errors first, exactly as fa_bwd reports them, before any CUDA call.
+  int rc = fa::validate_bwd(a, false);
   if (rc != FA_OK) return rc;
-  return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockmask, scratch,
-                kNoAllocScratchBytes, stream);
+  if (fa_bwd_workspace_bytes(B, H, N, d) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  rc = scratch_for_current_device(&scratch);
+  if (rc != FA_OK) return rc;
+  a.workspace = scratch;
+  a.workspace_bytes = kNoAllocScratchBytes;
+  return fa_bwd_ex(&a);
 }

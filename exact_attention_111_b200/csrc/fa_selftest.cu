@@ -1,4 +1,5 @@
-// fa_selftest.cu -- a diagnostic for the failure-detection path every kernel relies on.
+// fa_selftest.cu -- diagnostics: the failure-detection path every kernel relies on, and the
+// FMA-pipe exp2 the kernels use for part of their exponentials.
 //
 // Each kernel of the library bounds every mbarrier wait: past its time limit the wait
 // records FA_ERR_TIMEOUT in the device status word, raises the CTA's abort flag and
@@ -32,6 +33,17 @@ __global__ void __launch_bounds__(32) wait_timeout_probe(DevStatus st, int* wait
   }
 }
 
+// y[i] = 2^x[i] by the FMA-pipe polynomial the kernels use for part of their exponentials,
+// evaluated in pairs exactly as in the kernels (an odd tail pairs its last element with 0).
+__global__ void __launch_bounds__(256) exp2_poly_probe(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+  const float2 r = exp2_poly2(make_float2(a, b));
+  y[i] = r.x;
+  if (i + 1 < n) y[i + 1] = r.y;
+}
+
 }  // namespace
 }  // namespace fa
 
@@ -41,5 +53,12 @@ extern "C" int fa_selftest_wait_timeout(unsigned int limit_us, int* waited_ok, v
   if (status == nullptr) return FA_ERR_CUDA;
   fa::DevStatus st{status, (unsigned long long)limit_us * 1000ull};
   fa::wait_timeout_probe<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(st, waited_ok);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+extern "C" int fa_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 1 || x == nullptr || y == nullptr) return FA_ERR_INVALID_ARG;
+  const int pairs = (n + 1) / 2;
+  fa::exp2_poly_probe<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -376,9 +376,11 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
 
 // 2^x for a pair of x <= 0 on the FMA/ALU pipes, to take load off the special-function unit.
 // x = j + f with j = round(x) (added to the exponent field) and f in [-1/2, 1/2];
-// 2^f ~ 1 + c1 f + c2 f^2 + c3 f^3, max relative error 1.0e-4 (coefficients fitted by
-// exact_attention_111_b200/fit_exp2_poly.py).  x is clamped at -127, where the result is
-// exactly +0 (so -inf, a masked score, gives 0); x = 0 gives exactly 1.
+// 2^f ~ 1 + c1 f + c2 f^2 + c3 f^3, max relative error 1.0e-4 (coefficients: a minimax fit
+// of the relative error on [-1/2, 1/2] by Lawson's reweighted least squares, with the
+// constant term held at 1; tests/fit_exp2_poly.py reproduces them).  x is clamped at -127,
+// where the result is exactly +0 (so -inf, a masked score, gives 0); x = 0 gives exactly 1;
+// for x in (-127, -126) the result lies below 2^-126 (absolute error under 2^-126).
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kRound = 12582912.0f;            // 1.5 * 2^23: adding it rounds to an integer
   constexpr float c1 = 6.932829022e-01f, c2 = 2.422109544e-01f, c3 = 5.500892922e-02f;

@@ -24,6 +24,10 @@
  *   - The caller allocates and owns every buffer.  Inputs are read only.
  *   - Return value: FA_OK, or an fa_status error.  Argument errors return before anything
  *     is launched.  FA_ERR_CUDA means a CUDA runtime call failed at launch time.
+ *   - The library caches, per device ordinal, the device addresses of its own device
+ *     variables (the status word, fa_bwd_noalloc's array) for the life of the process, so it
+ *     must not be used across cudaDeviceReset (or any other teardown of a device's primary
+ *     context): after one, the cached addresses are stale.
  */
 #ifndef FA_B200_H_
 #define FA_B200_H_
@@ -70,6 +74,10 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  * Bytes of device workspace fa_bwd needs for this shape (fp32 dQ accumulator plus two
  * fp32 per-row vectors padded to whole 128-row tiles, each part 256-byte aligned).
  * Pure host arithmetic; returns 0 for invalid sizes.
+ * (NeurIPS22 summary, "核心方法 / Backward recomputation": the backward keeps O(N d) state
+ * besides its inputs -- the per-row statistics and one dQ accumulator -- never an N x N
+ * matrix; this is that state's size: B*H*N*(4*d) + 2 * B*H*ceil(N/128)*128*4 bytes, rounded
+ * up per part to 256 bytes.)
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -89,7 +97,13 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            int B, int H, int N, int d, float scale, int causal, const uint8_t* blockmask,
            void* workspace, size_t workspace_bytes, void* stream);
 
-/* General forms: element type, optional fp32 O output, optional tile visit log. */
+/*
+ * General forms of fa_fwd / fa_bwd (the same operation, "核心方法"; the pages fix no calling
+ * convention): element type bf16 or fp16, optional fp32 O output, optional tile visit log
+ * (the evidence that block-sparse skipping, "核心方法 / Block-sparse 扩展", computed exactly
+ * the kept tiles), per-kernel timing events, and the modes below (dropout, deterministic
+ * backward).  Errors as fa_fwd / fa_bwd.
+ */
 typedef struct {
   const void* q; const void* k; const void* v;
   void* o;                 /* bf16/fp16 like q, or fp32 when o_fp32 != 0            */
@@ -167,7 +181,10 @@ size_t fa_bwd_workspace_bytes_ex(int B, int H, int N, int d, int deterministic);
  * Synchronises `stream`, then reads and clears the device status word that kernels set
  * when a bounded wait expires (FA_ERR_TIMEOUT) or a deterministic backward meets a partial
  * outside its range (FA_ERR_RANGE).  Returns FA_OK, FA_ERR_TIMEOUT, FA_ERR_RANGE or
- * FA_ERR_CUDA.
+ * FA_ERR_CUDA.  FA_ERR_CUDA also stands for a kernel that found its own launch state
+ * unusable (its dynamic shared memory not 1024-byte aligned) and did no work; the device
+ * records such states under codes of its own, which are never returned as they are.
+ * (No counterpart in the pages: failure reporting of this library.)
  */
 int fa_check_status(void* stream);
 
@@ -190,8 +207,13 @@ int fa_check_status(void* stream);
  *   - returns FA_ERR_WORKSPACE, launching nothing, when fa_bwd_workspace_bytes(B, H, N, d)
  *     exceeds FA_NOALLOC_SCRATCH_BYTES (roughly B*H*N*(4*d + 8) bytes must fit in 64 MiB);
  *   - allocates nothing: no cudaMalloc / cudaFree and no allocating library routine;
- *   - the first call on a device looks up the array's device address for that device
- *     (cudaGetSymbolAddress); make that first call before any stream capture;
+ *   - the first call on a device does a one-time set-up there: the CUDA runtime loads the
+ *     library's device code lazily, so that call loads the code that holds the array, which
+ *     commits its FA_NOALLOC_SCRATCH_BYTES of device memory, and looks up the array's device
+ *     address (cudaGetSymbolAddress).  Make that first call at start-up, before any stream
+ *     capture and before device memory is frozen or exhausted; every later call allocates
+ *     nothing at all;
+ *   - argument errors are those of fa_bwd and come back before any CUDA call;
  *   - every call on a device shares the one array, which keeps the last call's contents
  *     (the backward rewrites all of it that it reads, so nothing needs clearing); calls that
  *     overlap on the GPU -- other streams or host threads -- race on it, so the caller
@@ -340,7 +362,18 @@ int fa_fwd_fp8(const fa_fwd_fp8_args* args);
  */
 int fa_selftest_wait_timeout(unsigned int limit_us, int* waited_ok, void* stream);
 
-/* Static human-readable name of a status code. */
+/*
+ * Diagnostic (no counterpart in the pages): y[i] = 2^x[i] for i < n, evaluated by the
+ * polynomial the kernels use for part of their exponentials to take load off the
+ * special-function unit (the FlashAttention-2 wiki, "最小化非矩阵运算", counts these
+ * non-matmul operations as the cost to cut).  x and y are device fp32 arrays of n elements.
+ * Claimed accuracy: relative error <= 1.1e-4 for x in [-126, 0]; exactly 1 at x = 0;
+ * exactly +0 for x <= -127 and for x = -inf; below 2^-126 in absolute value for x in
+ * (-127, -126).  One launch on `stream`; FA_ERR_INVALID_ARG for n < 1 or a NULL pointer.
+ */
+int fa_selftest_exp2_poly(const float* x, float* y, int n, void* stream);
+
+/* Static human-readable name of a status code (no counterpart in the pages). */
 const char* fa_status_string(int status);
 
 /* Number of kernel launches made by the last successful fa_fwd / fa_bwd call (any form) on this

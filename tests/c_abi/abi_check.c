@@ -69,6 +69,14 @@ int main(void) {
   }
   CHECK(fa_selftest_wait_timeout(0, NULL, NULL) == FA_ERR_INVALID_ARG);
 
+  /* fa_bwd_noalloc: fa_bwd's argument errors, before any CUDA call; then its size limit */
+  CHECK(fa_bwd_noalloc(NULL, fake, fake, fake, (const float*)fake, fake, fake, fake, fake, 1, 1, 128, 64, 0.125f, 0,
+                       NULL, NULL) == FA_ERR_INVALID_ARG);
+  CHECK(fa_bwd_noalloc(fake, fake, fake, fake, (const float*)fake, fake, fake, fake, fake, 1, 1, 128, 80, 0.125f, 0,
+                       NULL, NULL) == FA_ERR_UNSUPPORTED);
+  CHECK(fa_bwd_noalloc(fake, fake, fake, fake, (const float*)fake, fake, fake, fake, fake, 64, 16, 16384, 128,
+                       0.125f, 0, NULL, NULL) == FA_ERR_WORKSPACE);
+
   if (failures == 0) printf("c abi ok\n");
   return failures;
 }

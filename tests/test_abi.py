@@ -288,3 +288,42 @@ def test_fp8_workspace_and_argument_errors(L):
 def test_selftest_argument_errors(L):
     assert L.fa_selftest_wait_timeout(0, None, None) == fa.FA_ERR_INVALID_ARG
     assert L.fa_selftest_wait_timeout(1000001, None, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_noalloc_argument_errors_come_first(L):
+    """fa_bwd_noalloc reports fa_bwd's argument errors before any CUDA call (so also on a
+    host with no GPU), and refuses shapes whose workspace exceeds its fixed array."""
+    def call(ptr=FAKE, B=1, H=1, N=128, d=64, scale=0.125, lse=None):
+        p = ptr
+        return L.fa_bwd_noalloc(p, p, p, p, p if lse is None else lse, p, p, p, p, B, H, N, d,
+                                ctypes.c_float(scale), 0, None, None)
+    assert call(ptr=None) == fa.FA_ERR_INVALID_ARG
+    assert call(ptr=FAKE + 8) == fa.FA_ERR_INVALID_ARG
+    assert call(N=0) == fa.FA_ERR_INVALID_ARG
+    assert call(scale=0.0) == fa.FA_ERR_INVALID_ARG
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    # an oversized shape with NULL pointers is an argument error, as in fa_bwd
+    assert call(ptr=None, B=64, H=16, N=16384, d=128) == fa.FA_ERR_INVALID_ARG
+    # valid pointers but a workspace beyond the 64 MiB array: refused, nothing launched
+    assert fa.fa_bwd_workspace_bytes(64, 16, 16384, 128) > 64 << 20
+    assert call(B=64, H=16, N=16384, d=128) == fa.FA_ERR_WORKSPACE
+
+
+def test_device_status_codes_are_disjoint_from_public_codes():
+    """The kernels' status-word codes (csrc/fa_internal.h) share no value with the public
+    fa_status codes (include/fa.h), and fa_check_status translates each one by name."""
+    hdr = open(os.path.join(ROOT, "include", "fa.h")).read()
+    public = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(FA_(?:OK|ERR_\w+))\s*=\s*(\d+)", hdr)}
+    assert public["FA_ERR_RANGE"] == 6 and public["FA_ERR_TIMEOUT"] == 4
+    internal = open(os.path.join(ROOT, "exact_attention_111_b200", "csrc", "fa_internal.h")).read()
+    m = re.search(r"enum\s*:\s*int\s*\{([^}]*kDevTimeout[^}]*)\}", internal)
+    dev = {k: int(v, 0) for k, v in re.findall(r"(kDev\w+)\s*=\s*(0x[0-9a-fA-F]+|\d+)", m.group(1))}
+    assert dev["kDevOk"] == 0
+    nonzero = {k: v for k, v in dev.items() if k != "kDevOk"}
+    assert not set(nonzero.values()) & set(public.values())
+    host = open(os.path.join(ROOT, "exact_attention_111_b200", "csrc", "fa_host.cu")).read()
+    body = re.search(r"int status_from_device_word\(int v\) \{(.*?)\n\}", host, flags=re.S).group(1)
+    assert "case kDevTimeout: return FA_ERR_TIMEOUT;" in body
+    assert "case kDevRange: return FA_ERR_RANGE;" in body
+    assert "default: return FA_ERR_CUDA;" in body          # kDevBadState and anything else
+    assert "return status_from_device_word(v);" in host

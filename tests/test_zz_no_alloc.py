@@ -65,3 +65,30 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     p = t.data_ptr()
     rc = L.fa_bwd_noalloc(p, p, p, p, p, p, p, p, p, 1, 64, 16384, 128, 0.088, 0, None, None)
     assert rc == fa.FA_ERR_WORKSPACE
+
+
+def test_noalloc_calls_after_the_first_take_no_device_memory():
+    """The first call on a device is its set-up (the runtime loads the code holding the fixed
+    array, which commits the array, and the array's address is looked up).  Every later call
+    must leave the device's free memory exactly as it was: cudaMemGetInfo (torch.cuda.
+    mem_get_info) reads the same before and after it, and torch's allocator holds no more."""
+    P.ensure_built()
+    L = fa.lib()
+    stream = torch.cuda.current_stream().cuda_stream
+    B, H, N, d = 1, 2, 640, 64
+    inp = make_inputs(B, H, N, d, 41)
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "dout"))
+    o, lse = fa.attention_forward(q, k, v, causal=False)
+    got = [torch.empty_like(q) for _ in range(3)]
+    assert _c_call(L, q, k, v, o, lse, do, *got, B, H, N, d, d ** -0.5, False, None, stream) == fa.FA_OK
+    fa.fa_check_status()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for _ in range(2):
+        assert _c_call(L, q, k, v, o, lse, do, *got, B, H, N, d, d ** -0.5, False, None, stream) == fa.FA_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"free device memory changed by {free0 - free1} bytes"
+    assert torch.cuda.memory_allocated() == alloc0
+    fa.fa_check_status()
