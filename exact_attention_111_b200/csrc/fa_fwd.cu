@@ -7,19 +7,28 @@
 // ("Backward recomputation": the forward saves O and the softmax normalisation).
 //
 // One CTA owns two 128-row query tiles of one (b, h) head (256 rows), so every K/V tile
-// it loads feeds two score tiles.  Warp roles (320 threads):
-//   warps 0-3  softmax group 0: query tile 0, one row per thread (TMEM lanes 0..127)
-//   warps 4-7  softmax group 1: query tile 1
-//   warp  8    TMA producer: Q once, then the K/V ring (no multicast)
-//   warp  9    MMA issuer (one elected thread) and TMEM allocator
+// it loads feeds two score tiles.  Warp roles (512 threads, four warpgroups):
+//   warps 0-3    softmax group 0: query tile 0, one row per thread (TMEM lanes 0..127)
+//   warps 4-7    softmax group 1: query tile 1
+//   warps 8-11   correction: O_q <- alpha O_q in TMEM for both query tiles, one row per thread
+//   warp  12     TMA producer: Q once, then the K/V ring (no multicast)
+//   warp  13     MMA issuer (one elected thread) and TMEM allocator
+//   warps 14-15  idle (they complete the producer / MMA warpgroup)
+// setmaxnreg moves registers from the correction and producer / MMA warpgroups to the
+// softmax warpgroups, which hold a whole 128-score row each.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 [256+d, 256+2d).
 // (The one-query-tile layout of FwdCfg<D, 1>, used for short d = 64 sequences: softmax warps
-// 0-3, producer warp 4, MMA warp 5, 256 columns with S [0,128) and O [128,128+d).)
+// 0-3 that also rescale O, producer warp 4, MMA warp 5, 256 columns with S [0,128) and O
+// [128,128+d).)
 // P (16-bit) is written over the first 64 columns of its S tile and consumed from TMEM by
 // the PV MMA.  Per key tile u the MMA thread issues, for each query tile q that keeps u:
 //   O_q += P_q(prev) V(prev)   then   S_q = Q_q K(u)ᵀ   (commit -> s_full[q]),
-// so completion of S_q(u) also guarantees O_q holds every earlier PV product: the softmax
-// group may rescale O_q in place before releasing P_q(u).  The row max is refreshed whenever
+// so completion of S_q(u) also guarantees O_q holds every earlier PV product.  Once the
+// softmax group has the row maxima of S_q(u) it publishes the factors alpha = 2^(m_old - m_new);
+// the correction warps rescale O_q while the softmax group exponentiates, and the PV product
+// of tile u waits for both P_q(u) and the rescaled O_q.  This moves the rescale -- work that is
+// not a matrix product (FlashAttention-2 wiki, "最小化非矩阵运算") -- off the softmax's
+// critical path.  The row max is refreshed whenever
 // it grows, so the largest probability of a row is exactly 1 when it is rounded to 16 bits
 // (a stale max would leave it anywhere in [1, 2^k) and add up to 2^-8 relative rounding on the
 // dominant term of peaked rows).
@@ -44,7 +53,7 @@ namespace fa {
 namespace {
 
 // kQ query tiles per CTA.  kQ = 2 (the default): two softmax groups share every K/V tile,
-// 320 threads, all 512 TMEM columns, one CTA per SM.  kQ = 1 (d = 64, short sequences): one
+// 512 threads, all 512 TMEM columns, one CTA per SM.  kQ = 1 (d = 64, short sequences): one
 // softmax group, 192 threads, 256 TMEM columns and a 2-stage ring, so two CTAs fit on an SM
 // and one's start-up and epilogue overlap the other's tiles.
 template <int D, int kQ>
@@ -54,29 +63,47 @@ struct FwdCfg {
   static constexpr int kPanelBytes = kTile * 128;        // 128 rows x 128 bytes
   static constexpr int kStages = (kQ == 1) ? 2 : (D == 64) ? 4 : 2;   // K/V ring depth
   static constexpr int kSmemTiles = kQ * kTileBytes + 2 * kStages * kTileBytes;
-  static constexpr int kThreads = 128 * kQ + 64;
-  static constexpr int kLoadWarp = 4 * kQ, kMmaWarp = 4 * kQ + 1;
+  // kQ = 2: a correction warpgroup (warps 8-11) rescales O in TMEM while the softmax warps go
+  // on exponentiating; 16 warps, registers rebalanced per warpgroup with setmaxnreg.
+  static constexpr bool kCorr = (kQ == 2);
+  static constexpr int kThreads = kCorr ? 512 : 192;
+  static constexpr int kCorrWarp = 8;
+  static constexpr int kLoadWarp = kCorr ? 12 : 4, kMmaWarp = kCorr ? 13 : 5;
   static constexpr int kTmemCols = (kQ == 2) ? 512 : 256;
   static constexpr int kOCol = 128 * kQ;                 // first O column (S tiles before it)
   // exp2 pairs per 8 evaluated by polynomial on the FMA pipe instead of the SFU
   static constexpr int kPolyOf8 = (D == 64) ? 2 : 0;
+  // Registers per thread (kCorr): 128 at launch (65536 / 512), then softmax warpgroups 176,
+  // the correction warpgroup 88 and the load / MMA warpgroup 72 (the split with no spills at
+  // d = 128).  The shares add up to exactly the launch's 512 x 128, so every setmaxnreg.inc
+  // is satisfied.
+  static constexpr int kLaunchRegs = 128, kRegSoftmax = 176, kRegCorr = 88, kRegOther = 72;
+  static_assert(!kCorr || 8 * 32 * kRegSoftmax + 4 * 32 * kRegCorr + 4 * 32 * kRegOther <= kThreads * kLaunchRegs,
+                "register shares exceed the launch allocation");
 };
 
 struct FwdShared {
   uint64_t q_full;
   uint64_t k_full[4], v_full[4], kv_empty[4];
   uint64_t s_full[2], p_full[2];
+  uint64_t alpha_full[2], o_ready[2];   // softmax -> correction -> MMA (kCorr)
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
   int n_union;
   int n_q[2];
+  float alpha[2][kTile];                // per-row O rescale factor of the current tile (kCorr)
 };
+
+template <int N>
+__device__ __forceinline__ void reg_alloc_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void reg_alloc_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
 constexpr float kLn2 = 0.693147180559945309f;
 
 template <int D, bool kFp16, bool kDrop, int kQ>
-__global__ void __launch_bounds__(128 * kQ + 64, kQ == 2 ? 1 : 2)
+__global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
   using C = FwdCfg<D, kQ>;
@@ -111,6 +138,8 @@ __global__ void __launch_bounds__(128 * kQ + 64, kQ == 2 ? 1 : 2)
     for (int q = 0; q < kQ; ++q) {
       mbar_init(&sh.s_full[q], 1);
       mbar_init(&sh.p_full[q], 128);
+      mbar_init(&sh.alpha_full[q], 128);
+      mbar_init(&sh.o_ready[q], 128);
     }
     mbar_init(&sh.mma_done, 1);
     sh.abort_flag = 0;
@@ -153,6 +182,10 @@ __global__ void __launch_bounds__(128 * kQ + 64, kQ == 2 ? 1 : 2)
   const uint32_t tmem = sh.tmem_base;
   const int nu = sh.n_union;
 
+  // Each role's register share is set by its whole warpgroup at the top of the role's own
+  // branch (kCorr): softmax up to kRegSoftmax, correction and load / MMA down.
+  if (warp >= C::kLoadWarp) {
+  if constexpr (C::kCorr) reg_alloc_dec<C::kRegOther>();
   if (warp == C::kLoadWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && nu > 0) {
@@ -209,6 +242,9 @@ __global__ void __launch_bounds__(128 * kQ + 64, kQ == 2 ? 1 : 2)
               v_ready = true;
             }
             if (!mbar_wait(&sh.p_full[q], npv & 1, abort_flag, st)) return false;
+            if constexpr (C::kCorr) {     // O_q rescaled for this tile by the correction warps
+              if (!mbar_wait(&sh.o_ready[q], npv & 1, abort_flag, st)) return false;
+            }
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk) {
@@ -247,8 +283,54 @@ __global__ void __launch_bounds__(128 * kQ + 64, kQ == 2 ? 1 : 2)
       mbar_wait_drain(&sh.mma_done, 0, st);
     }
     __syncwarp();
+  }
+  } else if (C::kCorr && warp >= C::kCorrWarp) {
+    // ------------------------------------------------------------------ correction warpgroup
+    // For every tile a query tile keeps, in list order: wait for its softmax group to publish
+    // the per-row factors alpha = 2^(m_old - m_new), rescale that tile's O rows in TMEM (only
+    // warps where some row's max grew), and release O to the MMA warp.  The factor is known
+    // after the row max, long before P is, so this runs beside the softmax's exponentials.
+    // O_q then holds every earlier PV product: completion of S_q(u), which the softmax
+    // waited for before publishing, implies completion of PV_q(u-1) issued before it.
+    if constexpr (C::kCorr) reg_alloc_dec<C::kRegCorr>();
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    int cq[2] = {0, 0};
+    bool ok = true;
+    for (int u = 0; u < nu && ok; ++u) {
+      const int e = list[u];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (!((e >> (16 + q)) & 1)) continue;
+        ok = mbar_wait(&sh.alpha_full[q], cq[q] & 1, abort_flag, st);
+        if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+        const float al = sh.alpha[q][r];
+        if (cq[q] > 0 && __any_sync(0xffffffffu, al != 1.f)) {
+          tc_fence_after();
+          const uint32_t tO = tmem + C::kOCol + q * D + lane_off;
+#pragma unroll
+          for (int cc = 0; cc < D; cc += 32) {
+            uint32_t o[32];
+            tmem_ld32_sync(tO + cc, o);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float2 x = mul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), make_float2(al, al));
+              o[i] = __float_as_uint(x.x);
+              o[i + 1] = __float_as_uint(x.y);
+            }
+            tmem_st32(tO + cc, o);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(&sh.o_ready[q]);
+        ++cq[q];
+      }
+    }
   } else {
     // ------------------------------------------------------------------ softmax groups
+    if constexpr (C::kCorr) reg_alloc_inc<C::kRegSoftmax>();
     const int q = warp >> 2;
     const int wq = warp & 3;                        // TMEM lane quarter of this warp
     const int row_local = wq * 32 + lane;
@@ -306,6 +388,10 @@ __global__ void __launch_bounds__(128 * kQ + 64, kQ == 2 ? 1 : 2)
         resc = (c > 0);
         m = mx2;
       }
+      if constexpr (C::kCorr) {                     // hand the O rescale to the correction warps
+        sh.alpha[q][row_local] = alpha;
+        mbar_arrive(&sh.alpha_full[q]);
+      }
       const float mneg = (m == -INFINITY) ? 0.f : -m;
       const float2 sl2v = make_float2(sl2, sl2), mnegv = make_float2(mneg, mneg);
       // P = 2^(s*scale*log2e - m) in pairs (packed fp32 FMA), row sum over four packed
@@ -343,8 +429,9 @@ __global__ void __launch_bounds__(128 * kQ + 64, kQ == 2 ? 1 : 2)
       const float2 a0123 = add2(a01, a23);
       const float sum0 = a0123.x, sum1 = a0123.y;
       l = l * alpha + (sum0 + sum1);
-      // O <- alpha O for the rows whose max grew (O holds every earlier PV product: see above)
-      if (__any_sync(0xffffffffu, resc)) {
+      // O <- alpha O for the rows whose max grew (O holds every earlier PV product: see above);
+      // with a correction warpgroup that work is theirs
+      if (!C::kCorr && __any_sync(0xffffffffu, resc)) {
         const float f = resc ? alpha : 1.f;
 #pragma unroll
         for (int cc = 0; cc < D; cc += 32) {
@@ -427,6 +514,18 @@ cudaError_t launch_fwd_q(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   auto kern = a.drop.t > 0 ? fwd_kernel<D, kFp16, true, kQ> : fwd_kernel<D, kFp16, false, kQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  if constexpr (C::kCorr) {
+    // setmaxnreg.inc waits until the block's launch registers cover every warpgroup's share;
+    // refuse to launch a build whose register count differs from the one the shares assume.
+    static int regs = 0;
+    if (regs == 0) {
+      cudaFuncAttributes fa_attr;
+      e = cudaFuncGetAttributes(&fa_attr, kern);
+      if (e != cudaSuccess) return e;
+      regs = fa_attr.numRegs;
+    }
+    if (regs != C::kLaunchRegs) return cudaErrorInvalidConfiguration;
+  }
   const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.n_units) * static_cast<unsigned>(a.n_splits);
   kern<<<grid, C::kThreads, smem, s>>>(tq, tk, tv, a);
   return cudaGetLastError();
