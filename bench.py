@@ -301,13 +301,20 @@ class StepSetup:
         self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
         self.dq, self.dk, self.dv = (torch.empty_like(self.d[n]) for n in ("q", "k", "v"))
         self.det = bool(args.deterministic)
-        self.wsb = fa.fa_bwd_workspace_bytes_ex(B, H, N, D, self.det)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        # the workloads whose heads are too few to fill the GPU also split the backward's query
+        # ranges (not combinable with the deterministic mode)
+        self.qsplits = (fa.fa_bwd_splitq_choose(B, H, N, w.causal, sms)
+                        if w.fwd_splits is not None and not self.det else 0)
+        if args.bwd_splits is not None:
+            self.qsplits = args.bwd_splits
+        self.wsb = (fa.fa_bwd_workspace_bytes_split(B, H, N, D, self.qsplits) if self.qsplits > 1
+                    else fa.fa_bwd_workspace_bytes_ex(B, H, N, D, self.det))
         self.ws = torch.empty(self.wsb, dtype=torch.uint8, device=dev)
         self.stream = torch.cuda.current_stream(dev)
         self.splits = None
         if w.fwd_splits is not None:
-            self.splits = w.fwd_splits or fa.fa_splitkv_choose(
-                B, H, N, w.causal, torch.cuda.get_device_properties(dev).multi_processor_count)
+            self.splits = w.fwd_splits or fa.fa_splitkv_choose(B, H, N, w.causal, sms)
             self.wsfb = fa.fa_fwd_splitkv_workspace_bytes(B, H, N, D, self.splits)
             self.wsf = torch.empty(self.wsfb, dtype=torch.uint8, device=dev)
         self.pdrop, self.dseed = float(args.dropout), 0x5EED
@@ -332,7 +339,8 @@ class StepSetup:
         fa, w = self.fa, self.w
         fa.fa_bwd_ex(q, k, v, o_, lse_, do_, dq_, dk_, dv_, w.B, w.H, w.N, w.d, w.scale, w.causal, self.mask,
                      fa.FA_BF16, None, self.ws, self.wsb, self.stream, ev0, ev1,
-                     deterministic=self.det, dropout_p=self.pdrop, dropout_seed=self.dseed)
+                     deterministic=self.det, dropout_p=self.pdrop, dropout_seed=self.dseed,
+                     query_splits=self.qsplits)
         self.launches += fa.fa_last_launch_count()
 
     def step(self, ev=None):
@@ -470,6 +478,7 @@ def run_ours(args, w, world, rank, local):
     e2e_ms, h2d, d2h = time_e2e(st, e2e_steps, world)
     e2e_value = aggregate_tflops(world, r["step_flops"], e2e_steps, e2e_ms)
     main_splits = st.splits
+    main_qsplits = st.qsplits
     del st
     torch.cuda.empty_cache()
 
@@ -513,6 +522,7 @@ def run_ours(args, w, world, rank, local):
         "config": dict(workload_config(w, world),
                        **({"fwd_splits": main_splits, "fwd": "fa_fwd_splitkv (split forward + LSE merge, both inside "
                                                           "the fwd timing)"} if main_splits is not None else {}),
+                       **({"bwd_query_splits": main_qsplits} if main_qsplits > 1 else {}),
                        **({"deterministic_bwd": "int64 fixed-point dQ accumulation"} if st_det(args) else {}),
                        **({"dropout_p": args.dropout,
                            "dropout": "fused, Philox4x32-10 mask regenerated in the backward"}
@@ -654,6 +664,9 @@ def main():
     ap.add_argument("--fwd-splits", type=int, default=None,
                     help="forward through fa_fwd_splitkv with this many key ranges (0: chosen for the "
                          "GPU; default: the workload's own setting)")
+    ap.add_argument("--bwd-splits", type=int, default=None,
+                    help="backward with each key tile's query range cut into this many ranges "
+                         "(default: chosen for the GPU on the split-KV workloads, else none)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="fused dropout probability in both passes (default 0: none)")
     ap.add_argument("--fp8", action="store_true",

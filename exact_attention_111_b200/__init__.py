@@ -3,7 +3,7 @@
 The binding marshals arguments only; every step of the computation runs in the CUDA
 kernels behind the C ABI of ``include/fa.h``.  The C entry points are mirrored one to one
 (``fa_fwd``, ``fa_bwd``, ``fa_fwd_ex``, ``fa_bwd_ex``, ``fa_bwd_workspace_bytes``,
-``fa_bwd_workspace_bytes_ex``, ``fa_bwd_noalloc``, ``fa_fwd_partial``, ``fa_lse_merge``, ``fa_fwd_splitkv``,
+``fa_bwd_workspace_bytes_ex``, ``fa_bwd_workspace_bytes_split``, ``fa_bwd_splitq_choose``, ``fa_bwd_noalloc``, ``fa_fwd_partial``, ``fa_lse_merge``, ``fa_fwd_splitkv``,
 ``fa_fwd_splitkv_workspace_bytes``, ``fa_splitkv_choose``, ``fa_fwd_fp8``, ``fa_fwd_fp8_workspace_bytes``, ``fa_selftest_wait_timeout``, ``fa_selftest_exp2_poly``, ``fa_check_status``,
 ``fa_status_string``, ``fa_last_launch_count``); they take torch tensors (or raw device
 addresses as ints).  ``attention_forward`` / ``attention_backward`` /
@@ -24,7 +24,7 @@ __all__ = [
     "attention_forward", "attention_backward", "FlashAttention", "FA_BF16", "FA_FP16", "FA_FP32",
     "fa_fwd_partial", "fa_lse_merge", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes",
     "fa_splitkv_choose", "attention_forward_splitkv", "attention_forward_partial", "lse_merge",
-    "FA_MAX_PARTS", "fa_bwd_workspace_bytes_ex", "FA_ERR_RANGE", "fa_fwd_fp8", "fa_fwd_fp8_workspace_bytes",
+    "FA_MAX_PARTS", "fa_bwd_workspace_bytes_ex", "fa_bwd_workspace_bytes_split", "fa_bwd_splitq_choose", "FA_ERR_RANGE", "fa_fwd_fp8", "fa_fwd_fp8_workspace_bytes",
     "attention_forward_fp8", "fa_selftest_wait_timeout", "fa_selftest_exp2_poly",
 ]
 
@@ -58,7 +58,7 @@ class BwdArgs(ctypes.Structure):
                 ("blockmask", _vp), ("dtype", _i), ("visit_log", _vp),
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("stream", _vp),
                 ("main_start_event", _vp), ("main_stop_event", _vp), ("deterministic", _i),
-                ("dropout_p", _f), ("dropout_seed", ctypes.c_ulonglong)]
+                ("dropout_p", _f), ("dropout_seed", ctypes.c_ulonglong), ("query_splits", _i)]
 
 
 class PartialArgs(ctypes.Structure):
@@ -102,6 +102,10 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
     L.fa_bwd_workspace_bytes_ex.argtypes = [_i, _i, _i, _i, _i]
     L.fa_bwd_workspace_bytes_ex.restype = ctypes.c_size_t
+    L.fa_bwd_workspace_bytes_split.argtypes = [_i, _i, _i, _i, _i]
+    L.fa_bwd_workspace_bytes_split.restype = ctypes.c_size_t
+    L.fa_bwd_splitq_choose.argtypes = [_i, _i, _i, _i, _i]
+    L.fa_bwd_splitq_choose.restype = _i
     L.fa_check_status.argtypes = [_vp]
     L.fa_check_status.restype = _i
     L.fa_status_string.argtypes = [_i]
@@ -169,6 +173,14 @@ def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
 
 def fa_bwd_workspace_bytes_ex(B: int, H: int, N: int, d: int, deterministic: bool) -> int:
     return lib().fa_bwd_workspace_bytes_ex(B, H, N, d, int(bool(deterministic)))
+
+
+def fa_bwd_workspace_bytes_split(B: int, H: int, N: int, d: int, query_splits: int) -> int:
+    return lib().fa_bwd_workspace_bytes_split(B, H, N, d, int(query_splits))
+
+
+def fa_bwd_splitq_choose(B: int, H: int, N: int, causal: bool, num_sms: int) -> int:
+    return lib().fa_bwd_splitq_choose(B, H, N, int(bool(causal)), num_sms)
 
 
 def fa_check_status(stream=None):
@@ -268,12 +280,13 @@ def _event(e):
 
 def fa_bwd_ex(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal=False, blockmask=None,
               dtype=FA_BF16, visit_log=None, workspace=None, workspace_bytes=0, stream=None,
-              main_start_event=None, main_stop_event=None, deterministic=False, dropout_p=0.0, dropout_seed=0):
+              main_start_event=None, main_stop_event=None, deterministic=False, dropout_p=0.0, dropout_seed=0,
+              query_splits=0):
     a = BwdArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
                 _ptr(dv), B, H, N, d, scale, int(bool(causal)), _ptr(blockmask), dtype,
                 _ptr(visit_log), _ptr(workspace), workspace_bytes, _stream(stream),
                 _event(main_start_event), _event(main_stop_event), int(bool(deterministic)),
-                float(dropout_p), int(dropout_seed))
+                float(dropout_p), int(dropout_seed), int(query_splits))
     _check(lib().fa_bwd_ex(ctypes.byref(a)), "fa_bwd_ex")
 
 
@@ -385,14 +398,16 @@ def attention_forward_fp8(q8, k8, v8, descale_q, descale_k, descale_v, causal=Fa
 
 def attention_backward(q, k, v, o, lse, dout, causal=False, blockmask=None, scale=None,
                        workspace=None, visit_log=None, stream=None, deterministic=False, dropout_p=0.0,
-                       dropout_seed=0):
+                       dropout_seed=0, query_splits=0):
     """Returns (dQ, dK, dV) for the gradient ``dout`` of O.  ``deterministic``: bitwise
-    repeatable dQ through the int64 fixed-point accumulator (include/fa.h)."""
+    repeatable dQ through the int64 fixed-point accumulator; ``query_splits`` S >= 2: each key
+    tile's query range cut into S ranges (include/fa.h)."""
     import torch
     _check_qkv(q, k, v, o, dout)
     B, H, N, d = q.shape
     scale = (1.0 / d ** 0.5) if scale is None else scale
-    nbytes = fa_bwd_workspace_bytes_ex(B, H, N, d, deterministic)
+    nbytes = (fa_bwd_workspace_bytes_split(B, H, N, d, query_splits) if query_splits > 1
+              else fa_bwd_workspace_bytes_ex(B, H, N, d, deterministic))
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     dq = torch.empty_like(q)
@@ -400,7 +415,7 @@ def attention_backward(q, k, v, o, lse, dout, causal=False, blockmask=None, scal
     dv = torch.empty_like(v)
     fa_bwd_ex(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, blockmask,
               _dtype_code(q), visit_log, workspace, workspace.numel(), stream, deterministic=deterministic,
-              dropout_p=dropout_p, dropout_seed=dropout_seed)
+              dropout_p=dropout_p, dropout_seed=dropout_seed, query_splits=query_splits)
     return dq, dk, dv
 
 

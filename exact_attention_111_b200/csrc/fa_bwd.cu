@@ -80,6 +80,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreArgs a) {
         z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
         z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      if (a.dk_acc != nullptr) {
+        float4* zk = reinterpret_cast<float4*>(a.dk_acc + off);
+        float4* zv = reinterpret_cast<float4*>(a.dv_acc + off);
+        zk[0] = zk[1] = zv[0] = zv[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
     if (a.dq_fix != nullptr && active) {       // every row of the padded accumulator, 4 x 16 bytes
       const long long tile = (long long)bh * (a.Np / 128) + i / 128;
@@ -105,17 +110,26 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreArgs a) {
 // bwd_post
 // ------------------------------------------------------------------------------------
 template <bool kFp16>
+__device__ __forceinline__ void convert8(const float* acc, void* out, long long t, float f) {
+  const float4* src = reinterpret_cast<const float4*>(acc) + 2 * t;
+  const float4 x = src[0], y = src[1];
+  uint4 w;
+  w.x = pack2<kFp16>(x.x * f, x.y * f);
+  w.y = pack2<kFp16>(x.z * f, x.w * f);
+  w.z = pack2<kFp16>(y.x * f, y.y * f);
+  w.w = pack2<kFp16>(y.z * f, y.w * f);
+  reinterpret_cast<uint4*>(out)[t] = w;
+}
+
+template <bool kFp16>
 __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdPostArgs a) {
   const long long n8 = a.n_elems / 8;
   for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n8; t += (long long)gridDim.x * blockDim.x) {
-    const float4* src = reinterpret_cast<const float4*>(a.dq_acc) + 2 * t;
-    const float4 x = src[0], y = src[1];
-    uint4 w;
-    w.x = pack2<kFp16>(x.x * a.scale, x.y * a.scale);
-    w.y = pack2<kFp16>(x.z * a.scale, x.w * a.scale);
-    w.z = pack2<kFp16>(y.x * a.scale, y.y * a.scale);
-    w.w = pack2<kFp16>(y.z * a.scale, y.w * a.scale);
-    reinterpret_cast<uint4*>(a.dq)[t] = w;
+    convert8<kFp16>(a.dq_acc, a.dq, t, a.scale);
+    if (a.dk_acc != nullptr) {                 // query-range splits: dK and dV from their accumulators
+      convert8<kFp16>(a.dk_acc, a.dk, t, a.scale);
+      convert8<kFp16>(a.dv_acc, a.dv, t, 1.f);
+    }
   }
 }
 
@@ -235,9 +249,9 @@ __device__ __forceinline__ uint64_t drop_bits(const Dropout& dr, int j, int wq, 
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
-// Next step k' >= k whose query tile the key tile j keeps (T when none).
-__device__ __forceinline__ int next_kept(int k, int j, int T, int causal, const uint8_t* mask) {
-  for (; k < T; ++k) {
+// Next step k' in [k, k_end) whose query tile the key tile j keeps (k_end when none).
+__device__ __forceinline__ int next_kept(int k, int j, int k_end, int T, int causal, const uint8_t* mask) {
+  for (; k < k_end; ++k) {
     const int i = rot_tile(k, j, T);
     if (causal && i < j) continue;
     if (mask != nullptr && __ldg(mask + (size_t)i * T + j) == 0) continue;
@@ -264,8 +278,12 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
   // CTAs resident together share a few heads, so those heads' Q / dO tiles and fp32 dQ
   // accumulator rows stay in L2 (ordering by key tile across all heads thrashed L2); within
   // a group, key tile 0 (the heaviest under causal masking) goes first.
-  int bh, j;
-  cta_order(blockIdx.x, a.BH, a.T, a.group_heads, bh, j);
+  int bh, j, slot;
+  cta_order(blockIdx.x, a.BH, a.T * a.q_splits, a.group_heads, bh, slot);
+  j = slot / a.q_splits;
+  // query-range split of this CTA: visiting steps k in [k_begin, k_end)
+  const int k_begin = (slot - j * a.q_splits) * a.q_chunk;
+  const int k_end = min(a.T, k_begin + a.q_chunk);
   const DevStatus st{a.status, a.timeout_ns};
   volatile int* abort_flag = &sh.abort_flag;
   const bool aligned = (smem_addr(smem) & 1023u) == 0;
@@ -295,8 +313,8 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
-  const int k_first = next_kept(0, j, a.T, a.causal, a.blockmask);
-  const bool any = aligned && k_first < a.T;
+  const int k_first = next_kept(k_begin, j, k_end, a.T, a.causal, a.blockmask);
+  const bool any = aligned && k_first < k_end;
 
   if (warp == kLoadW) {
     // ------------------------------------------------------------------ TMA producer
@@ -311,7 +329,7 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
         tma_load_3d(smem + C::oV + p * C::kPanelBytes, &tm_v, &sh.kv_full, p * 64, j * kTile, bh);
       }
       int c = 0;
-      for (int k = k_first; k < a.T; k = next_kept(k + 1, j, a.T, a.causal, a.blockmask), ++c) {
+      for (int k = k_first; k < k_end; k = next_kept(k + 1, j, k_end, a.T, a.causal, a.blockmask), ++c) {
         const int i = rot_tile(k, j, a.T);
         const int s = c % C::kStages;
         if (c >= C::kStages && !mbar_wait(&sh.q_empty[s], ((c / C::kStages) - 1) & 1, abort_flag, st)) break;
@@ -374,10 +392,10 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
         issue_s(0);
         if (a.visit != nullptr) atomicAdd(&a.visit[((size_t)bh * a.T + rot_tile(k_first, j, a.T)) * a.T + j], 1);
         issue_dp(0);
-        for (int k = k_first; k < a.T; ++c) {
+        for (int k = k_first; k < k_end; ++c) {
           const int s = c % C::kStages;
-          const int k_next = next_kept(k + 1, j, a.T, a.causal, a.blockmask);
-          const bool more = k_next < a.T;
+          const int k_next = next_kept(k + 1, j, k_end, a.T, a.causal, a.blockmask);
+          const bool more = k_next < k_end;
           const int i_next = more ? rot_tile(k_next, j, a.T) : 0;
           const uint32_t qb = aQ + s * C::kTileBytes, dob = aDO + s * C::kTileBytes;
           // dV += Pᵀ dO(c)   (Pᵀ read from tensor memory)
@@ -529,7 +547,7 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
       return true;
     };
     if (any) {
-      for (int k = k_first; k < a.T; k = next_kept(k + 1, j, a.T, a.causal, a.blockmask), ++c) {
+      for (int k = k_first; k < k_end; k = next_kept(k + 1, j, k_end, a.T, a.causal, a.blockmask), ++c) {
         const int i = rot_tile(k, j, a.T);
         const int s = c % C::kStages;
         uint32_t keep_lo = 0u, keep_hi = 0u;        // dropout keep bits of this row's 64 columns
@@ -657,7 +675,25 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
     // Epilogue: group 0 writes dV, group 1 writes scale * dK, one key row per thread.
     if (ok) ok = mbar_wait(&sh.mma_done, 0, abort_flag, st);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && g < 2) {
+    if (ok && g < 2 && a.q_splits > 1) {
+      // query-range split: add this range's partial (dV, unscaled dK) into the fp32 accumulators
+      if (c > 0) {
+        tc_fence_after();
+        const uint32_t tA = tmem + (g == 0 ? C::tDV : C::tDK) + lane_off;
+        float* acc = (g == 0 ? a.dv_acc : a.dk_acc) + ((size_t)bh * a.N + key) * D;
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t v[32];
+          tmem_ld32_sync(tA + cc, v);
+          if (key_ok) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              red_add_v4(acc + cc + 4 * t, __uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
+                         __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3]));
+          }
+        }
+      }
+    } else if (ok && g < 2) {
       tc_fence_after();
       const size_t base = ((size_t)bh * a.N + key) * D;
       const uint32_t tA = tmem + (g == 0 ? C::tDV : C::tDK) + lane_off;
@@ -712,7 +748,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.T);
+  const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.T) * static_cast<unsigned>(a.q_splits);
   kern<<<grid, threads, C::kSmem, s>>>(tq, tk, tv, tdo, tdq, a);
   return cudaGetLastError();
 }

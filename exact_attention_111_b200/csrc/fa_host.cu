@@ -147,19 +147,26 @@ SplitLayout split_layout(int B, int H, int N, int d, int S) {
 }
 
 struct WsLayout {
-  size_t dq_acc, delta, lse2, total;
+  size_t dq_acc, delta, lse2, dk_acc, dv_acc, total;
 };
 
 // The dQ accumulator is fp32 [BH, N, d], or in deterministic mode int64 over whole tiles
-// [BH, Np, d] (tile-blocked, fix_index).
-WsLayout ws_layout(int B, int H, int N, int d, bool det = false) {
+// [BH, Np, d] (tile-blocked, fix_index).  With query-range splits (q_splits > 1) fp32 dK and
+// dV accumulators [BH, N, d] follow.
+WsLayout ws_layout(int B, int H, int N, int d, bool det = false, int q_splits = 1) {
   const size_t BH = (size_t)B * H;
   const size_t Np = (size_t)((N + kTile - 1) / kTile) * kTile;
   WsLayout w;
   w.dq_acc = 0;
   w.delta = det ? align256(BH * Np * d * 8) : align256(BH * N * d * 4);
   w.lse2 = w.delta + align256(BH * Np * 4);
-  w.total = w.lse2 + align256(BH * Np * 4);
+  w.dk_acc = w.lse2 + align256(BH * Np * 4);
+  w.dv_acc = w.dk_acc;
+  w.total = w.dk_acc;
+  if (q_splits > 1) {
+    w.dv_acc = w.dk_acc + align256(BH * N * d * 4);
+    w.total = w.dv_acc + align256(BH * N * d * 4);
+  }
   return w;
 }
 
@@ -204,8 +211,13 @@ int validate_bwd(const fa_bwd_args& x, bool check_workspace) {
     return FA_ERR_INVALID_ARG;
   Dropout drop{};
   if (!make_dropout(x.dropout_p, x.dropout_seed, &drop)) return FA_ERR_INVALID_ARG;
+  if (x.query_splits < 0 || x.query_splits > FA_MAX_PARTS) return FA_ERR_INVALID_ARG;
+  // the split ranges add dK / dV partials in fp32 in whatever order they finish
+  if (x.query_splits > 1 && x.deterministic) return FA_ERR_UNSUPPORTED;
+  const int T = (x.N + kTile - 1) / kTile;
+  if ((long long)x.B * x.H * T * (x.query_splits > 1 ? x.query_splits : 1) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   if (check_workspace) {
-    const WsLayout w = ws_layout(x.B, x.H, x.N, x.d, x.deterministic != 0);
+    const WsLayout w = ws_layout(x.B, x.H, x.N, x.d, x.deterministic != 0, x.query_splits);
     if (!x.workspace || !aligned(x.workspace, 256) || x.workspace_bytes < w.total) return FA_ERR_WORKSPACE;
   }
   return FA_OK;
@@ -245,6 +257,45 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
 size_t fa_bwd_workspace_bytes_ex(int B, int H, int N, int d, int deterministic) {
   if (check_shape(B, H, N, d, 1.f, FA_BF16) != FA_OK) return 0;
   return ws_layout(B, H, N, d, deterministic != 0).total;
+}
+
+size_t fa_bwd_workspace_bytes_split(int B, int H, int N, int d, int query_splits) {
+  if (check_shape(B, H, N, d, 1.f, FA_BF16) != FA_OK) return 0;
+  if (query_splits < 0 || query_splits > FA_MAX_PARTS) return 0;
+  return ws_layout(B, H, N, d, false, query_splits).total;
+}
+
+int fa_bwd_splitq_choose(int B, int H, int N, int causal, int num_sms) {
+  if (B < 1 || H < 1 || N < 1 || N > FA_MAX_SEQLEN || num_sms < 1) return 0;
+  const long long T = (N + kTile - 1) / kTile;
+  const long long BH = (long long)B * H;
+  const long long total = BH * (causal ? T * (T + 1) / 2 : T * T);   // (key, query) tile pairs
+  const long long avg = (total + num_sms - 1) / num_sms;
+  int best = 1;
+  long long best_cost = -1;
+  for (int S = 1; S <= FA_MAX_PARTS; ++S) {
+    const long long chunk = (T + S - 1) / S;       // query steps per range
+    if (S > 1 && chunk < 4) break;
+    const long long s_eff = (T + chunk - 1) / chunk;
+    if (s_eff < S) continue;                        // the same cut as a smaller S
+    // CTAs with work: under causal masking key tile j keeps T - j steps, so range s is empty
+    // for the key tiles past T - s * chunk
+    long long ctas = 0;
+    for (long long sr = 0; sr < s_eff; ++sr) ctas += causal ? (T - sr * chunk) : T;
+    ctas *= BH;
+    const long long waves = (ctas + num_sms - 1) / num_sms;
+    // Finishing time in tiles: CTAs of equal length (no causal mask) run in whole waves; causal
+    // CTAs range from `chunk` tiles down to one, and the heaviest-first order packs them to about
+    // the average load per SM, but no faster than the longest.  Plus about two tiles of fixed
+    // cost per CTA in each wave.
+    const long long span = causal ? (chunk > avg ? chunk : avg) : waves * chunk;
+    const long long cost = span + 2 * waves;
+    if (best_cost < 0 || 10 * cost < 9 * best_cost) {   // a larger count must win by 10 %
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
 }
 
 int fa_fwd_ex(const fa_fwd_args* p) {
@@ -303,7 +354,8 @@ int fa_bwd_ex(const fa_bwd_args* p) {
   Dropout drop{};
   make_dropout(x.dropout_p, x.dropout_seed, &drop);
   const bool det = x.deterministic != 0;
-  const WsLayout w = ws_layout(x.B, x.H, x.N, x.d, det);
+  const int qs = x.query_splits > 1 ? x.query_splits : 1;
+  const WsLayout w = ws_layout(x.B, x.H, x.N, x.d, det, qs);
   const bool fp16 = x.dtype == FA_FP16;
   const int BH = x.B * x.H;
   const int T = (x.N + kTile - 1) / kTile;
@@ -328,6 +380,9 @@ int fa_bwd_ex(const fa_bwd_args* p) {
   BwdPreArgs pre{};
   pre.o = x.o; pre.dout = x.dout; pre.lse = x.lse;
   pre.delta = delta; pre.lse2 = lse2; pre.dq_acc = dq_acc; pre.dq_fix = dq_fix;
+  float* dk_acc = qs > 1 ? reinterpret_cast<float*>(ws + w.dk_acc) : nullptr;
+  float* dv_acc = qs > 1 ? reinterpret_cast<float*>(ws + w.dv_acc) : nullptr;
+  pre.dk_acc = dk_acc; pre.dv_acc = dv_acc;
   pre.N = x.N; pre.Np = Np; pre.BH = BH; pre.d = x.d;
   if (launch_bwd_pre(pre, fp16, s) != cudaSuccess) return FA_ERR_CUDA;
 
@@ -335,7 +390,10 @@ int fa_bwd_ex(const fa_bwd_args* p) {
   b.delta = delta; b.lse2 = lse2; b.dq_acc = dq_acc; b.dq_fix = dq_fix; b.dk = x.dk; b.dv = x.dv;
   b.blockmask = x.blockmask; b.visit = x.visit_log; b.status = status; b.timeout_ns = kWaitLimitNs;
   b.N = x.N; b.Np = Np; b.BH = BH; b.T = T; b.causal = x.causal != 0;
-  b.group_heads = group_heads_for(BH, T);
+  b.q_splits = qs;
+  b.q_chunk = (T + qs - 1) / qs;
+  b.dk_acc = dk_acc; b.dv_acc = dv_acc;
+  b.group_heads = group_heads_for(BH, T * qs);
   b.scale = x.scale;
   b.scale_log2 = (float)((double)x.scale * 1.4426950408889634);
   b.drop = drop;
@@ -347,6 +405,7 @@ int fa_bwd_ex(const fa_bwd_args* p) {
 
   BwdPostArgs post{};
   post.dq_acc = dq_acc; post.dq_fix = dq_fix; post.dq = x.dq; post.n_elems = (long long)BH * x.N * x.d;
+  post.dk_acc = dk_acc; post.dv_acc = dv_acc; post.dk = x.dk; post.dv = x.dv;
   post.N = x.N; post.Np = Np; post.BH = BH; post.d = x.d; post.scale = x.scale;
   if (launch_bwd_post(post, fp16, s) != cudaSuccess) return FA_ERR_CUDA;
   t_last_launches = 3;

@@ -71,6 +71,8 @@ struct BwdPreArgs {
   float* dq_acc;            // [BH, N, d] fp32, zeroed here (when dq_fix is null)
   long long* dq_fix;        // deterministic mode: int64 fixed-point accumulator (tile-blocked,
                             // see fix_index), zeroed here; null otherwise
+  float* dk_acc;            // query-range splits: fp32 dK / dV accumulators [BH, N, d], zeroed
+  float* dv_acc;            // here; null otherwise
   int N, Np, BH, d;
 };
 
@@ -88,6 +90,13 @@ struct BwdArgs {
   int N, Np, BH, T;
   int group_heads;          // CTAs are ordered in groups of this many heads (see cta_order)
   int causal;
+  // Query-range splits: key tile j's kept query tiles, in its visiting order k = 0, 1, ..., are
+  // cut into q_splits ranges of q_chunk steps, one CTA per (head, key tile, range).  With
+  // q_splits > 1 each CTA adds its partial dK (unscaled) and dV into dk_acc / dv_acc (fp32)
+  // instead of writing dk / dv, and the post pass converts them.
+  int q_splits, q_chunk;
+  float* dk_acc;
+  float* dv_acc;
   float scale;              // multiplies dK (dQ is scaled in the post pass)
   float scale_log2;
   Dropout drop;
@@ -97,6 +106,10 @@ struct BwdPostArgs {
   const float* dq_acc;      // [BH, N, d]
   const long long* dq_fix;  // deterministic mode: the int64 accumulator (else null)
   void* dq;                 // [BH, N, d] 16-bit
+  const float* dk_acc;      // query-range splits: the fp32 dK / dV accumulators (else null);
+  const float* dv_acc;      // dk = 16-bit(scale * dk_acc), dv = 16-bit(dv_acc)
+  void* dk;
+  void* dv;
   long long n_elems;
   int N, Np, BH, d;
   float scale;

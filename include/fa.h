@@ -139,6 +139,9 @@ typedef struct {
                               must then hold fa_bwd_workspace_bytes_ex(..., 1) bytes    */
   float dropout_p;         /* exactly the forward's dropout_p and dropout_seed        */
   unsigned long long dropout_seed;
+  int query_splits;        /* 0 or 1: off; S >= 2: split each key tile's query range, see
+                              below (the workspace must then hold
+                              fa_bwd_workspace_bytes_split(..., S) bytes)               */
 } fa_bwd_args;
 
 int fa_fwd_ex(const fa_fwd_args* args);
@@ -176,6 +179,29 @@ int fa_bwd_ex(const fa_bwd_args* args);
  * Workspace bytes for either mode; fa_bwd_workspace_bytes(...) == ..._ex(..., 0).
  */
 size_t fa_bwd_workspace_bytes_ex(int B, int H, int N, int d, int deterministic);
+
+/*
+ * Query-range splits of the backward (fa_bwd_args.query_splits = S >= 2), its counterpart of the
+ * split-KV forward.  The FlashAttention-2 wiki ("改进并行性") spreads one head's work over the
+ * SMs because a small batch of long sequences otherwise leaves SMs idle.  The backward runs one
+ * CTA per (head, 128-key tile), and that CTA walks the key tile's query tiles; with few heads
+ * there are too few CTAs, and under causal masking key tile 0 walks all T query tiles while
+ * the last walks one.  With S splits each key tile's visited query tiles are cut into S ranges
+ * of ceil(T / S) steps, one CTA per (head, key tile, range).  Each range's dK and dV partials
+ * are added in fp32 into workspace accumulators and a final pass converts them, so:
+ *   - the result equals the unsplit one up to fp32 summation order (not bitwise);
+ *   - it does not combine with deterministic != 0 (FA_ERR_UNSUPPORTED);
+ *   - the workspace grows by two fp32 [B, H, N, d] accumulators:
+ *     fa_bwd_workspace_bytes_split(B, H, N, d, S) (== fa_bwd_workspace_bytes for S <= 1).
+ * 0 <= query_splits <= FA_MAX_PARTS, else FA_ERR_INVALID_ARG.
+ * fa_bwd_splitq_choose: host arithmetic, the S to use on a GPU with num_sms SMs: minimises the
+ * finishing time in tiles -- whole waves of equal ranges without causal masking, else
+ * max(longest range, average (key, query) tile pairs per SM) -- plus 2 per wave of CTAs, over
+ * 1 .. FA_MAX_PARTS with at least 4 steps per range; a larger S must win by 10 %.  Returns 1
+ * when the key tiles alone fill the GPU, 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_bytes_split(int B, int H, int N, int d, int query_splits);
+int fa_bwd_splitq_choose(int B, int H, int N, int causal, int num_sms);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word that kernels set

@@ -51,6 +51,12 @@ int main(void) {
   ba.workspace = (void*)(size_t)0x100000; ba.deterministic = 1;
   ba.workspace_bytes = fa_bwd_workspace_bytes_ex(1, 1, 128, 64, 1) - 1;
   CHECK(fa_bwd_ex(&ba) == FA_ERR_WORKSPACE);
+  ba.workspace_bytes = (size_t)1 << 30; ba.query_splits = 2;   /* splits and the deterministic mode */
+  CHECK(fa_bwd_ex(&ba) == FA_ERR_UNSUPPORTED);
+  ba.deterministic = 0; ba.query_splits = 65;
+  CHECK(fa_bwd_ex(&ba) == FA_ERR_INVALID_ARG);
+  CHECK(fa_bwd_workspace_bytes_split(1, 1, 128, 64, 2) == fa_bwd_workspace_bytes(1, 1, 128, 64) + 2 * 128 * 64 * 4);
+  CHECK(fa_bwd_splitq_choose(1, 1, 16384, 1, 148) == 3);
 
   memset(&f8, 0, sizeof f8);
   f8.q = f8.k = f8.v = fake; f8.o = fake; f8.lse = (float*)fake;

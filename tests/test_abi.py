@@ -327,3 +327,59 @@ def test_device_status_codes_are_disjoint_from_public_codes():
     assert "case kDevRange: return FA_ERR_RANGE;" in body
     assert "default: return FA_ERR_CUDA;" in body          # kDevBadState and anything else
     assert "return status_from_device_word(v);" in host
+
+
+def test_split_backward_workspace_and_arguments(L):
+    """Query-range splits: the workspace adds two fp32 [B, H, N, d] accumulators; S <= 1 is the
+    plain layout; S outside [0, 64] and S >= 2 with the deterministic mode are refused."""
+    a = lambda x: (x + 255) // 256 * 256
+    for B, H, N, d in ((1, 1, 16384, 128), (2, 3, 1000, 64)):
+        base = fa.fa_bwd_workspace_bytes(B, H, N, d)
+        assert fa.fa_bwd_workspace_bytes_split(B, H, N, d, 0) == base
+        assert fa.fa_bwd_workspace_bytes_split(B, H, N, d, 1) == base
+        assert fa.fa_bwd_workspace_bytes_split(B, H, N, d, 3) == base + 2 * a(B * H * N * d * 4)
+    assert fa.fa_bwd_workspace_bytes_split(1, 1, 128, 64, 65) == 0
+    ws = fa.fa_bwd_workspace_bytes_split(1, 1, 128, 64, 2)
+
+    def call(splits, det=0, wsb=ws):
+        b = fa.BwdArgs(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None,
+                       fa.FA_BF16, None, 0x100000, wsb, None, None, None, det, 0.0, 0, splits)
+        return L.fa_bwd_ex(ctypes.byref(b))
+    assert call(-1) == fa.FA_ERR_INVALID_ARG
+    assert call(65) == fa.FA_ERR_INVALID_ARG
+    assert call(2, det=1, wsb=1 << 30) == fa.FA_ERR_UNSUPPORTED
+    assert call(2, wsb=ws - 1) == fa.FA_ERR_WORKSPACE
+
+
+def splitq_choose_reference(B, H, N, causal, sms):
+    """The choice restated: minimise the finishing time (whole waves of equal ranges without a
+    causal mask, else max(longest range, average tile pairs per SM)) + 2 per wave of non-empty
+    CTAs over S = 1 .. 64 with at least 4 steps per range; a larger S must win by 10 %."""
+    T = -(-N // 128)
+    total = B * H * (T * (T + 1) // 2 if causal else T * T)
+    avg = -(-total // sms)
+    best, best_cost = 1, None
+    for S in range(1, 65):
+        chunk = -(-T // S)
+        if S > 1 and chunk < 4:
+            break
+        s_eff = -(-T // chunk)
+        if s_eff < S:
+            continue
+        ctas = B * H * sum((T - s * chunk) if causal else T for s in range(s_eff))
+        waves = -(-ctas // sms)
+        cost = (max(chunk, avg) if causal else waves * chunk) + 2 * waves
+        if best_cost is None or 10 * cost < 9 * best_cost:
+            best, best_cost = S, cost
+    return best
+
+
+def test_split_backward_choice(L):
+    assert fa.fa_bwd_splitq_choose(1, 1, 16384, True, 148) == 3
+    assert fa.fa_bwd_splitq_choose(1, 1, 16384, False, 148) == 1     # 128 equal CTAs: one wave already
+    assert fa.fa_bwd_splitq_choose(1, 32, 16384, True, 148) == 1     # the long-context batch fills the GPU
+    assert fa.fa_bwd_splitq_choose(64, 16, 1024, False, 148) == 1
+    assert fa.fa_bwd_splitq_choose(0, 1, 128, False, 148) == 0
+    for B, H, N, causal in ((1, 1, 16384, True), (1, 2, 8192, True), (2, 1, 4096, False), (1, 1, 1000, True),
+                            (1, 4, 32768, True), (3, 5, 777, False)):
+        assert fa.fa_bwd_splitq_choose(B, H, N, causal, 148) == splitq_choose_reference(B, H, N, causal, 148)
