@@ -84,7 +84,7 @@ struct FwdCfg {
 
 struct FwdShared {
   uint64_t q_full;
-  uint64_t k_full[4], v_full[4], kv_empty[4];
+  uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
   uint64_t s_full[2], p_full[2];
   uint64_t alpha_full[2], o_ready[2];   // softmax -> correction -> MMA (kCorr)
   uint64_t mma_done;
@@ -133,7 +133,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&sh.k_full[s], 1);
       mbar_init(&sh.v_full[s], 1);
-      mbar_init(&sh.kv_empty[s], 1);
+      mbar_init(&sh.k_empty[s], 1);
+      mbar_init(&sh.v_empty[s], 1);
     }
     for (int q = 0; q < kQ; ++q) {
       mbar_init(&sh.s_full[q], 1);
@@ -197,25 +198,32 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
       for (int q = 0; q < nq; ++q)
         for (int p = 0; p < C::kPanels; ++p)
           tma_load_3d(sQ + q * C::kTileBytes + p * C::kPanelBytes, &tm_q, &sh.q_full, p * 64, (qt0 + q) * kTile, bh);
-      int u = 0;
-      for (; u < nu; ++u) {
+      // K and V slots are released separately: a key tile's slot frees when the last S product
+      // that reads it completes, a full PV product earlier than its value tile's slot, so the
+      // next key tile is already resident when the MMA warp reaches it.
+      int nk = 0, nv = 0;                         // key / value tiles whose copy was started
+      for (int u = 0; u < nu; ++u) {
         const int s = u % C::kStages;
-        if (u >= C::kStages && !mbar_wait(&sh.kv_empty[s], ((u / C::kStages) - 1) & 1, abort_flag, st)) break;
+        const uint32_t ph = ((u / C::kStages) - 1) & 1;
         const int j = list[u] & 0xFFFF;
+        if (u >= C::kStages && !mbar_wait(&sh.k_empty[s], ph, abort_flag, st)) break;
         mbar_arrive_expect_tx(&sh.k_full[s], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
           tma_load_3d(sK + s * C::kTileBytes + p * C::kPanelBytes, &tm_k, &sh.k_full[s], p * 64, j * kTile, bh);
+        ++nk;
+        if (u >= C::kStages && !mbar_wait(&sh.v_empty[s], ph, abort_flag, st)) break;
         mbar_arrive_expect_tx(&sh.v_full[s], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
           tma_load_3d(sV + s * C::kTileBytes + p * C::kPanelBytes, &tm_v, &sh.v_full[s], p * 64, j * kTile, bh);
+        ++nv;
       }
       if (*abort_flag) {
         // Let every copy this thread started land before the CTA's shared memory goes away.
         mbar_wait_drain(&sh.q_full, 0, st);
-        for (int uu = (u > C::kStages ? u - C::kStages : 0); uu < u; ++uu) {
+        for (int uu = (nk > C::kStages ? nk - C::kStages : 0); uu < nk; ++uu)
           mbar_wait_drain(&sh.k_full[uu % C::kStages], (uu / C::kStages) & 1, st);
+        for (int uu = (nv > C::kStages ? nv - C::kStages : 0); uu < nv; ++uu)
           mbar_wait_drain(&sh.v_full[uu % C::kStages], (uu / C::kStages) & 1, st);
-        }
       }
     }
     __syncwarp();
@@ -234,8 +242,9 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
         const int sp = (u + C::kStages - 1) % C::kStages;
         const int sc = u % C::kStages;
         bool v_ready = false, k_ready = false;
-        // For query tile q: O_q += P_q V(u-1) if it kept tile u-1, then S_q = Q_q K(u)ᵀ if it keeps u.
-        auto step = [&](int q, int& npv) -> bool {
+        // Per iteration: O_0 += P_0 V(u-1), S_0 = Q_0 K(u)ᵀ, O_1 += P_1 V(u-1), S_1 = Q_1 K(u)ᵀ, each
+        // only where that query tile keeps the tile.
+        auto pv = [&](int q, int& npv) -> bool {
           if (u > 0 && ((ep >> (16 + q)) & 1)) {
             if (!v_ready) {
               if (!mbar_wait(&sh.v_full[sp], ((u - 1) / C::kStages) & 1, abort_flag, st)) return false;
@@ -253,6 +262,9 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
             }
             ++npv;
           }
+          return true;
+        };
+        auto sq = [&](int q) -> bool {
           if (u < nu && ((ec >> (16 + q)) & 1)) {
             if (!k_ready) {
               if (!mbar_wait(&sh.k_full[sc], (u / C::kStages) & 1, abort_flag, st)) return false;
@@ -272,8 +284,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
           }
           return true;
         };
-        ok = step(0, npv0) && (kQ == 1 || step(1, npv1));
-        if (u > 0 && ok) tc_commit(&sh.kv_empty[sp]);
+        ok = pv(0, npv0) && sq(0) && (kQ == 1 || pv(1, npv1));
+        if (u > 0 && ok) tc_commit(&sh.v_empty[sp]);       // V(u-1) free once its PV products are done
+        ok = ok && (kQ == 1 || sq(1));
+        if (u < nu && ok) tc_commit(&sh.k_empty[sc]);      // K(u) free once its S products are done
       }
       if (ok) {
         tc_commit(&sh.s_full[0]);   // final phase: every MMA into O_0 / O_1 has completed

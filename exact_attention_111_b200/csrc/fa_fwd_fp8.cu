@@ -54,7 +54,7 @@ constexpr float kLn2F8 = 0.693147180559945309f;
 
 struct F8Shared {
   uint64_t q_full;
-  uint64_t k_full[kF8Stages], v_full[kF8Stages], kv_empty[kF8Stages];
+  uint64_t k_full[kF8Stages], v_full[kF8Stages], k_empty[kF8Stages], v_empty[kF8Stages];
   uint64_t s_full[2], p_full[2];
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -145,7 +145,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < kF8Stages; ++s) {
       mbar_init(&sh.k_full[s], 1);
       mbar_init(&sh.v_full[s], 1);
-      mbar_init(&sh.kv_empty[s], 1);
+      mbar_init(&sh.k_empty[s], 1);
+      mbar_init(&sh.v_empty[s], 1);
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(&sh.s_full[q], 1);
@@ -198,22 +199,27 @@ __global__ void __launch_bounds__(320, 1)
       const int nq = (qt0 + 1 < a.T) ? 2 : 1;
       mbar_arrive_expect_tx(&sh.q_full, nq * kF8TileBytes);
       for (int q = 0; q < nq; ++q) tma_load_3d(sQ + q * kF8TileBytes, &tm_q, &sh.q_full, 0, (qt0 + q) * kTile, bh);
-      int u = 0;
-      for (; u < nu; ++u) {
+      // key and value slots are released separately (the key slot a PV product earlier)
+      int nk = 0, nv = 0;
+      for (int u = 0; u < nu; ++u) {
         const int s = u % kF8Stages;
-        if (u >= kF8Stages && !mbar_wait(&sh.kv_empty[s], ((u / kF8Stages) - 1) & 1, abort_flag, st)) break;
+        const uint32_t ph = ((u / kF8Stages) - 1) & 1;
         const int j = list[u] & 0xFFFF;
+        if (u >= kF8Stages && !mbar_wait(&sh.k_empty[s], ph, abort_flag, st)) break;
         mbar_arrive_expect_tx(&sh.k_full[s], kF8TileBytes);
         tma_load_3d(sK + s * kF8TileBytes, &tm_k, &sh.k_full[s], 0, j * kTile, bh);
+        ++nk;
+        if (u >= kF8Stages && !mbar_wait(&sh.v_empty[s], ph, abort_flag, st)) break;
         mbar_arrive_expect_tx(&sh.v_full[s], kF8TileBytes);
         tma_load_3d(sV + s * kF8TileBytes, &tm_vt, &sh.v_full[s], j * kTile, 0, bh);
+        ++nv;
       }
       if (*abort_flag) {
         mbar_wait_drain(&sh.q_full, 0, st);
-        for (int uu = (u > kF8Stages ? u - kF8Stages : 0); uu < u; ++uu) {
+        for (int uu = (nk > kF8Stages ? nk - kF8Stages : 0); uu < nk; ++uu)
           mbar_wait_drain(&sh.k_full[uu % kF8Stages], (uu / kF8Stages) & 1, st);
+        for (int uu = (nv > kF8Stages ? nv - kF8Stages : 0); uu < nv; ++uu)
           mbar_wait_drain(&sh.v_full[uu % kF8Stages], (uu / kF8Stages) & 1, st);
-        }
       }
     }
     __syncwarp();
@@ -230,8 +236,9 @@ __global__ void __launch_bounds__(320, 1)
         const int sp = (u + kF8Stages - 1) % kF8Stages;
         const int sc = u % kF8Stages;
         bool v_ready = false, k_ready = false;
-        // For query tile q: O_q += P_q Vᵀ(u-1)ᵀ if it kept tile u-1, then S_q = Q_q K(u)ᵀ.
-        auto step = [&](int q, int& npv) -> bool {
+        // Per iteration: O_0 += P_0 V(u-1), S_0 = Q_0 K(u)ᵀ, O_1 += P_1 V(u-1), S_1 = Q_1 K(u)ᵀ, each
+        // only where that query tile keeps the tile.
+        auto pv = [&](int q, int& npv) -> bool {
           if (u > 0 && ((ep >> (16 + q)) & 1)) {
             if (!v_ready) {
               if (!mbar_wait(&sh.v_full[sp], ((u - 1) / kF8Stages) & 1, abort_flag, st)) return false;
@@ -247,6 +254,9 @@ __global__ void __launch_bounds__(320, 1)
             }
             ++npv;
           }
+          return true;
+        };
+        auto sq = [&](int q) -> bool {
           if (u < nu && ((ec >> (16 + q)) & 1)) {
             if (!k_ready) {
               if (!mbar_wait(&sh.k_full[sc], (u / kF8Stages) & 1, abort_flag, st)) return false;
@@ -263,8 +273,10 @@ __global__ void __launch_bounds__(320, 1)
           }
           return true;
         };
-        ok = step(0, npv0) && step(1, npv1);
-        if (u > 0 && ok) tc_commit(&sh.kv_empty[sp]);
+        ok = pv(0, npv0) && sq(0) && pv(1, npv1);
+        if (u > 0 && ok) tc_commit(&sh.v_empty[sp]);       // V(u-1) free once its PV products are done
+        ok = ok && sq(1);
+        if (u < nu && ok) tc_commit(&sh.k_empty[sc]);      // K(u) free once its S products are done
       }
       if (ok) {
         tc_commit(&sh.s_full[0]);   // final phase: every MMA into O_0 / O_1 has completed
