@@ -63,12 +63,14 @@ struct FwdCfg {
   static constexpr int kPanelBytes = kTile * 128;        // 128 rows x 128 bytes
   static constexpr int kStages = (kQ == 1) ? 2 : (D == 64) ? 4 : 2;   // K/V ring depth
   static constexpr int kSmemTiles = kQ * kTileBytes + 2 * kStages * kTileBytes;
-  // kQ = 2: a correction warpgroup (warps 8-11) rescales O in TMEM while the softmax warps go
-  // on exponentiating; 16 warps, registers rebalanced per warpgroup with setmaxnreg.
-  static constexpr bool kCorr = (kQ == 2);
-  static constexpr int kThreads = kCorr ? 512 : 192;
+  // kQ = 2 at d = 128: a correction warpgroup (warps 8-11) rescales O in TMEM while the
+  // softmax warps go on exponentiating; 16 warps, registers rebalanced per warpgroup with
+  // setmaxnreg.  At d = 64 the rescale of 64 columns is cheap and the softmax warps keep it
+  // (measured: the correction warpgroup costs the d = 64 forward 5-16 %).
+  static constexpr bool kCorr = (kQ == 2 && D == 128);
+  static constexpr int kThreads = kCorr ? 512 : 128 * kQ + 64;
   static constexpr int kCorrWarp = 8;
-  static constexpr int kLoadWarp = kCorr ? 12 : 4, kMmaWarp = kCorr ? 13 : 5;
+  static constexpr int kLoadWarp = kCorr ? 12 : 4 * kQ, kMmaWarp = kCorr ? 13 : 4 * kQ + 1;
   static constexpr int kTmemCols = (kQ == 2) ? 512 : 256;
   static constexpr int kOCol = 128 * kQ;                 // first O column (S tiles before it)
   // exp2 pairs per 8 evaluated by polynomial on the FMA pipe instead of the SFU
