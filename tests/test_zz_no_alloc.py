@@ -9,6 +9,8 @@ alone in a fresh process."""
 
 from __future__ import annotations
 
+import gc
+
 import numpy as np
 import pytest
 import torch
@@ -71,7 +73,8 @@ def test_noalloc_calls_after_the_first_take_no_device_memory():
     """The first call on a device is its set-up (the runtime loads the code holding the fixed
     array, which commits the array, and the array's address is looked up).  Every later call
     must leave the device's free memory exactly as it was: cudaMemGetInfo (torch.cuda.
-    mem_get_info) reads the same before and after it, and torch's allocator holds no more."""
+    mem_get_info) reads the same before and after it, and torch's allocator holds no more
+    (it may hold less: tensors of earlier tests can be collected meanwhile)."""
     P.ensure_built()
     L = fa.lib()
     stream = torch.cuda.current_stream().cuda_stream
@@ -82,6 +85,7 @@ def test_noalloc_calls_after_the_first_take_no_device_memory():
     got = [torch.empty_like(q) for _ in range(3)]
     assert _c_call(L, q, k, v, o, lse, do, *got, B, H, N, d, d ** -0.5, False, None, stream) == fa.FA_OK
     fa.fa_check_status()
+    gc.collect()
     torch.cuda.synchronize()
     free0, _ = torch.cuda.mem_get_info()
     alloc0 = torch.cuda.memory_allocated()
@@ -90,5 +94,5 @@ def test_noalloc_calls_after_the_first_take_no_device_memory():
     torch.cuda.synchronize()
     free1, _ = torch.cuda.mem_get_info()
     assert free1 == free0, f"free device memory changed by {free0 - free1} bytes"
-    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.cuda.memory_allocated() <= alloc0
     fa.fa_check_status()
