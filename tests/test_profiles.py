@@ -26,6 +26,13 @@ def test_stored_traffic_is_published_only_for_the_current_sources():
             assert bench.stored_traffic(kernel, workload) == expect, f"{kernel} on {workload}"
 
 
+def test_default_workload_traffic_is_published():
+    """The dominant kernels of the default bench workload have a DRAM figure taken on the
+    current sources, so the bench line's roofline.traffic is not null."""
+    for kernel in ("fwd", "bwd_main"):
+        assert bench.stored_traffic(kernel, bench.DEFAULT_WORKLOAD) is not None, kernel
+
+
 def test_profile_summaries_are_text_and_small():
     for name in os.listdir(os.path.join(ROOT, "profiles")):
         p = os.path.join(ROOT, "profiles", name)
