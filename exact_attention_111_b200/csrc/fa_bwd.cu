@@ -187,9 +187,10 @@ struct BwdCfg {
 };
 
 constexpr int kBwdThreads = 320;   // 2 compute groups (8 warps), producer, MMA issuer
-// d = 64, default mode: four compute groups of 32 query columns (18 warps, 96 registers) instead
-// of two.  The twice as many warps hide the phase latencies that bound this kernel at d = 64
-// (measured backward main: +5 to +7 % from N = 512 to 16384, causal included).
+// d = 64, float dQ: four compute groups of 32 query columns (18 warps, 96 registers) instead of
+// two.  The twice as many warps hide the phase latencies that bound this kernel at d = 64
+// (measured backward main: +5 to +7 % from N = 512 to 16384, causal included; with dropout,
+// whose generator work they also share, +7 to +19 %).
 constexpr bool kBwdFourGroups = true;
 
 struct BwdBars {
@@ -249,6 +250,43 @@ __device__ __forceinline__ uint64_t drop_bits(const Dropout& dr, int j, int wq, 
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
+// The same for the 32 query columns q0 .. q0+31 of a four-group layout: lane L draws the calls
+// of columns 2 * (L % 16) + k (k = 0, 1) for the key block of its half-warp, words rotated by
+// L % 4; in round (k, q, s) a lane of word group w reads slot s from lane
+// 16 * half + 4q + ((w - s) mod 4), whose columns are 2 * (4q + ((w - s) mod 4)) + k: 32 shuffles
+// deliver each lane the byte of all 32 columns.  Bit c of the result is query q0 + c.
+__device__ __forceinline__ uint32_t drop_bits32(const Dropout& dr, int j, int wq, int lane, int q0, int bh) {
+  const int half = lane >> 4;
+  const uint32_t jb = static_cast<uint32_t>((j * kTile + wq * 32) >> 4) + half;
+  const int rot = lane & 3;
+  uint32_t R[2][4];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint4 w4 = philox4x32_10(make_uint4(jb, static_cast<uint32_t>(q0 + 2 * (lane & 15) + k),
+                                              static_cast<uint32_t>(bh), 0u), dr.seed_lo, dr.seed_hi);
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      const int idx = (sl + rot) & 3;
+      R[k][sl] = (idx & 2) ? ((idx & 1) ? w4.w : w4.z) : ((idx & 1) ? w4.y : w4.x);
+    }
+  }
+  const int w = (lane & 15) >> 2;
+  const int bsh = 8 * (lane & 3);
+  uint32_t bits = 0u;
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int sl = 0; sl < 4; ++sl) {
+        const int g4 = (w - sl) & 3;
+        const uint32_t x = __shfl_sync(0xffffffffu, R[k][sl], (half << 4) | (4 * q + g4));
+        const uint32_t bit = ((x >> bsh) & 0xFFu) >= dr.t ? 1u : 0u;
+        bits |= bit << (2 * (4 * q + g4) + k);
+      }
+  return bits;
+}
+
 // Next step k' in [k, k_end) whose query tile the key tile j keeps (k_end when none).
 __device__ __forceinline__ int next_kept(int k, int j, int k_end, int T, int causal, const uint8_t* mask) {
   for (; k < k_end; ++k) {
@@ -269,7 +307,7 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
   using C = BwdCfg<D>;
-  static_assert(kG == 2 || (kG == 4 && D == 64 && !kDet && !kDrop), "four groups: d = 64, default mode");
+  static_assert(kG == 2 || (kG == 4 && D == 64 && !kDet), "four groups: d = 64, float dQ");
   constexpr int kLoadW = 4 * kG, kMmaW = 4 * kG + 1;
   constexpr int kCols = kTile / kG;                 // query columns per compute group
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -550,11 +588,15 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
       for (int k = k_first; k < k_end; k = next_kept(k + 1, j, k_end, a.T, a.causal, a.blockmask), ++c) {
         const int i = rot_tile(k, j, a.T);
         const int s = c % C::kStages;
-        uint32_t keep_lo = 0u, keep_hi = 0u;        // dropout keep bits of this row's 64 columns
+        uint32_t keep_lo = 0u, keep_hi = 0u;        // dropout keep bits of this row's kCols columns
         if constexpr (kDrop) {
-          const uint64_t kb = drop_bits(a.drop, j, wq, lane, i * kTile + 64 * g, bh);
-          keep_lo = static_cast<uint32_t>(kb);
-          keep_hi = static_cast<uint32_t>(kb >> 32);
+          if constexpr (kCols == 64) {
+            const uint64_t kb = drop_bits(a.drop, j, wq, lane, i * kTile + 64 * g, bh);
+            keep_lo = static_cast<uint32_t>(kb);
+            keep_hi = static_cast<uint32_t>(kb >> 32);
+          } else {
+            keep_lo = drop_bits32(a.drop, j, wq, lane, i * kTile + kCols * g, bh);
+          }
         }
         ok = mbar_wait(&sh.q_full[s], (c / C::kStages) & 1, abort_flag, st) &&
              mbar_wait(&sh.s_full, c & 1, abort_flag, st);
@@ -602,7 +644,7 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
         if constexpr (kDrop) {
           // dV takes P o M: dropped columns 0, kept ones scaled (pk keeps the undropped P)
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
+          for (int h2 = 0; h2 < kCols / 32; ++h2) {
             uint32_t pd[16];
             const uint32_t kw = h2 == 0 ? keep_lo : keep_hi;
 #pragma unroll
@@ -611,7 +653,7 @@ __global__ void __launch_bounds__(128 * kG + 64, 1)
               pd[t] = pack2<kFp16>(((kw >> (2 * t)) & 1u) ? p.x * a.drop.scale : 0.f,
                                    ((kw >> (2 * t + 1)) & 1u) ? p.y * a.drop.scale : 0.f);
             }
-            tmem_st16(tS + 64 * g + 16 * h2, pd);
+            tmem_st16(tS + kCols * g + 16 * h2, pd);
           }
         } else {
           if constexpr (kCols == 64) tmem_st32(tS + 64 * g, pk);
@@ -750,8 +792,8 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                                   : (drop ? bwd_kernel<D, kFp16, false, true, 2> : bwd_kernel<D, kFp16, false, false, 2>);
   int threads = kBwdThreads;
   if constexpr (D == 64) {
-    if (kBwdFourGroups && a.dq_fix == nullptr && !drop) {
-      kern = bwd_kernel<D, kFp16, false, false, 4>;
+    if (kBwdFourGroups && a.dq_fix == nullptr) {
+      kern = drop ? bwd_kernel<D, kFp16, false, true, 4> : bwd_kernel<D, kFp16, false, false, 4>;
       threads = 4 * 128 + 64;
     }
   }

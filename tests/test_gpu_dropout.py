@@ -69,22 +69,25 @@ def test_forward_mask_is_bit_exact(B, H, N):
                 assert np.array_equal(kept[b, h], ref), (b, h, kt)
 
 
-def test_backward_mask_is_bit_exact():
-    """dO = identity on query rows 0..127 (zero elsewhere): dV[j, c] = (P o M)[c, j]."""
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_mask_is_bit_exact(d):
+    """dO = identity on query rows off .. off+d-1 (zero elsewhere): dV[j, c] = (P o M)[off + c, j].
+    d = 64 runs the four-group layout (32 query columns per group), d = 128 the two-group one."""
     P.ensure_built()
     B, H, N, p, seed = 2, 2, 384, 0.45, 987654321
-    inp = P.inputs(B, H, N, 128, seed=6100)
+    inp = P.inputs(B, H, N, d, seed=6100 + d)
     o, lse = _fwd(inp, False, None, p, seed)
-    do = torch.zeros((B, H, N, 128), dtype=torch.bfloat16)
-    do[:, :, :128] = torch.eye(128, dtype=torch.bfloat16)
-    inp2 = dict(inp)
-    inp2["dout"] = do
-    g = _bwd(inp2, o, lse, False, None, p, seed)
-    kept = (g["dv"].float() != 0).cpu().numpy()         # [B, H, N keys, 128 query rows]
-    for b in range(B):
-        for h in range(H):
-            ref = od.keep_mask(b * H + h, N, N, seed, p)[:128, :].T
-            assert np.array_equal(kept[b, h], ref), (b, h)
+    for off in range(0, 128, d):
+        do = torch.zeros((B, H, N, d), dtype=torch.bfloat16)
+        do[:, :, off:off + d] = torch.eye(d, dtype=torch.bfloat16)
+        inp2 = dict(inp)
+        inp2["dout"] = do
+        g = _bwd(inp2, o, lse, False, None, p, seed)
+        kept = (g["dv"].float() != 0).cpu().numpy()         # [B, H, N keys, d query rows]
+        for b in range(B):
+            for h in range(H):
+                ref = od.keep_mask(b * H + h, N, N, seed, p)[off:off + d, :].T
+                assert np.array_equal(kept[b, h], ref), (b, h, off)
 
 
 CASES = [
