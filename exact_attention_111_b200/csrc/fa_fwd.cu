@@ -52,10 +52,11 @@
 namespace fa {
 namespace {
 
-// kQ query tiles per CTA.  kQ = 2 (the default): two softmax groups share every K/V tile,
-// 512 threads, all 512 TMEM columns, one CTA per SM.  kQ = 1 (d = 64, short sequences): one
-// softmax group, 192 threads, 256 TMEM columns and a 2-stage ring, so two CTAs fit on an SM
-// and one's start-up and epilogue overlap the other's tiles.
+// kQ query tiles per CTA.  kQ = 2 (d = 128, and d = 64 with dropout past 8 key tiles): two
+// softmax groups share every K/V tile, one CTA per SM (at d = 128 with a correction warpgroup,
+// 512 threads, all 512 TMEM columns).  kQ = 1 (d = 64): one softmax group, 192 threads, 256
+// TMEM columns and a 2-stage ring, so two CTAs fit on an SM and one's start-up and epilogue
+// overlap the other's tiles.
 template <int D, int kQ>
 struct FwdCfg {
   static constexpr int kPanels = D / 64;                 // 64-element (128-byte) swizzle panels
@@ -73,6 +74,15 @@ struct FwdCfg {
   static constexpr int kLoadWarp = kCorr ? 12 : 4 * kQ, kMmaWarp = kCorr ? 13 : 4 * kQ + 1;
   static constexpr int kTmemCols = (kQ == 2) ? 512 : 256;
   static constexpr int kOCol = 128 * kQ;                 // first O column (S tiles before it)
+  // One query tile at d = 64 leaves TMEM columns for P of its own (after S and O): S(u+1) is
+  // then issued as soon as the softmax has read S(u) instead of after the PV product that
+  // reads P(u), which takes that MMA pair off the softmax's chain; the softmax instead waits
+  // for PV(u) before it rescales O and stores P(u+1).  Measured forward: +13.5 % at N = 1024,
+  // +5 % at N = 512; with two query tiles (which also have the columns) it lost 5-9 %, and
+  // the dropout variant (kernel-side switch) spills and lost 27 %.
+  static constexpr bool kEarlyS = (D == 64 && kQ == 1);
+  static constexpr int kPCol = kQ * (128 + D);           // first P column (kEarlyS)
+  static_assert(!kEarlyS || kPCol + 64 * kQ <= kTmemCols, "P columns exceed the allocation");
   // exp2 pairs per 8 evaluated by polynomial on the FMA pipe instead of the SFU
   static constexpr int kPolyOf8 = (D == 64) ? 2 : 0;
   // Registers per thread (kCorr): 128 at launch (65536 / 512), then softmax warpgroups 176,
@@ -89,6 +99,7 @@ struct FwdShared {
   uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
   uint64_t s_full[2], p_full[2];
   uint64_t alpha_full[2], o_ready[2];   // softmax -> correction -> MMA (kCorr)
+  uint64_t s_free[2], pv_done[2];       // S_q read by the softmax / PV_q product done (kEarlyS)
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -109,6 +120,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
   using C = FwdCfg<D, kQ>;
+  constexpr bool kES = C::kEarlyS && !kDrop;   // P in its own TMEM columns, early S issue
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ FwdShared sh;
 
@@ -143,6 +155,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
       mbar_init(&sh.p_full[q], 128);
       mbar_init(&sh.alpha_full[q], 128);
       mbar_init(&sh.o_ready[q], 128);
+      mbar_init(&sh.s_free[q], 128);
+      mbar_init(&sh.pv_done[q], 1);
     }
     mbar_init(&sh.mma_done, 1);
     sh.abort_flag = 0;
@@ -238,6 +252,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
       const uint32_t idesc_pv = idesc_f16(128, D, kFp16, false, true);
       const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
       int npv0 = 0, npv1 = 0;                     // PV products issued per query tile
+      int ns[2] = {0, 0};                         // S products issued per query tile
       for (int u = 0; u <= nu && ok; ++u) {
         const int ep = (u > 0) ? list[u - 1] : 0;
         const int ec = (u < nu) ? list[u] : 0;
@@ -257,11 +272,14 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
               if (!mbar_wait(&sh.o_ready[q], npv & 1, abort_flag, st)) return false;
             }
             tc_fence_after();
+            // P_q: its own columns (kEarlyS) or over S_q
+            const uint32_t tPq = kES ? tmem + C::kPCol + 64 * q : tmem + q * 128;
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk) {
               const uint64_t bdesc = smem_desc_sw128(aV + sp * C::kTileBytes + kk * 2048, C::kPanelBytes, 1024);
-              mma_ts(tmem + C::kOCol + q * D, tmem + q * 128 + kk * 8, bdesc, idesc_pv, (npv > 0 || kk > 0) ? 1u : 0u);
+              mma_ts(tmem + C::kOCol + q * D, tPq + kk * 8, bdesc, idesc_pv, (npv > 0 || kk > 0) ? 1u : 0u);
             }
+            if constexpr (kES) tc_commit(&sh.pv_done[q]);
             ++npv;
           }
           return true;
@@ -273,6 +291,13 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
               tc_fence_after();
               k_ready = true;
             }
+            if constexpr (kES) {            // the softmax has read S_q's previous tile
+              if (ns[q] > 0) {
+                if (!mbar_wait(&sh.s_free[q], (ns[q] - 1) & 1, abort_flag, st)) return false;
+                tc_fence_after();
+              }
+            }
+            ++ns[q];
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
@@ -286,10 +311,19 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
           }
           return true;
         };
-        ok = pv(0, npv0) && sq(0) && (kQ == 1 || pv(1, npv1));
-        if (u > 0 && ok) tc_commit(&sh.v_empty[sp]);       // V(u-1) free once its PV products are done
-        ok = ok && (kQ == 1 || sq(1));
-        if (u < nu && ok) tc_commit(&sh.k_empty[sc]);      // K(u) free once its S products are done
+        if constexpr (kES) {
+          // S_0(u), S_1(u) as soon as the softmax groups have read the previous S, then the PV
+          // products of tile u-1 as their P arrive
+          ok = sq(0) && (kQ == 1 || sq(1));
+          if (u < nu && ok) tc_commit(&sh.k_empty[sc]);
+          ok = ok && pv(0, npv0) && (kQ == 1 || pv(1, npv1));
+          if (u > 0 && ok) tc_commit(&sh.v_empty[sp]);
+        } else {
+          ok = pv(0, npv0) && sq(0) && (kQ == 1 || pv(1, npv1));
+          if (u > 0 && ok) tc_commit(&sh.v_empty[sp]);     // V(u-1) free once its PV products are done
+          ok = ok && (kQ == 1 || sq(1));
+          if (u < nu && ok) tc_commit(&sh.k_empty[sc]);    // K(u) free once its S products are done
+        }
       }
       if (ok) {
         tc_commit(&sh.s_full[0]);   // final phase: every MMA into O_0 / O_1 has completed
@@ -355,6 +389,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + q * 128 + lane_off;
     const uint32_t tO = tmem + C::kOCol + q * D + lane_off;
+    const uint32_t tP = kES ? tmem + C::kPCol + 64 * q + lane_off : tS;   // P_q's columns
     const float sl2 = a.scale_log2;
     float m = -INFINITY;   // running max of scale*log2(e)*s over this row
     float l = 0.f;         // running sum of 2^(scale*log2(e)*s - m)
@@ -376,6 +411,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
       tmem_wait_ld();
 #pragma unroll
       for (int cq = 0; cq < 4; ++cq) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cq]));
+      if constexpr (kES) {                   // S_q's columns may take the next tile
+        tc_fence_before();
+        mbar_arrive(&sh.s_free[q]);
+      }
       float s[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
@@ -410,6 +449,15 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
       }
       const float mneg = (m == -INFINITY) ? 0.f : -m;
       const float2 sl2v = make_float2(sl2, sl2), mnegv = make_float2(mneg, mneg);
+      if constexpr (kES) {
+        // PV_q of the previous kept tile must be done: it reads the P columns about to be
+        // rewritten, and O must hold it before the rescale below
+        if (c > 0) {
+          ok = mbar_wait(&sh.pv_done[q], (c - 1) & 1, abort_flag, st);
+          if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+          tc_fence_after();
+        }
+      }
       // P = 2^(s*scale*log2e - m) in pairs (packed fp32 FMA), row sum over four packed
       // accumulators; P stored to TMEM in quarters of 32 keys as soon as each is packed.
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -439,7 +487,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
             pk[i] = pack2<kFp16>(p.x, p.y);
           }
         }
-        tmem_st16(tS + 16 * h, pk);
+        tmem_st16(tP + 16 * h, pk);
       }
       const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
       const float2 a0123 = add2(a01, a23);
@@ -562,9 +610,10 @@ cudaError_t launch_fwd_q(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   return cudaGetLastError();
 }
 
-// Single-tile CTAs pay off while a CTA's start-up and epilogue are large next to its key
-// tiles: d = 64 with at most kSingleMaxTiles key tiles per CTA (measured forward: +9 % at 4
-// tiles, +1.5 % at 8, -2 % at 16 and slower beyond).
+// At d = 64 the one-query-tile layout, with its early S issue, is the faster forward at every
+// length measured (N = 512 to 16384, causal too: +13 to +19 % over two query tiles from
+// N = 2048 on).  With dropout it has no early issue, and pays off only while a CTA's start-up
+// and epilogue are large next to its key tiles: up to kSingleMaxTiles key tiles.
 constexpr int kSingleMaxTiles = 8;
 
 template <int D, bool kFp16>
@@ -572,7 +621,7 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          cudaStream_t s) {
   if constexpr (D == 64) {
     const int tiles = min(a.Tk, a.split_tiles);
-    if (tiles <= kSingleMaxTiles && (long long)a.BH * a.T * a.n_splits <= 0x7fffffffLL)
+    if ((a.drop.t == 0 || tiles <= kSingleMaxTiles) && (long long)a.BH * a.T * a.n_splits <= 0x7fffffffLL)
       return launch_fwd_q<D, kFp16, 1>(tq, tk, tv, a, s);
   }
   return launch_fwd_q<D, kFp16, 2>(tq, tk, tv, a, s);
