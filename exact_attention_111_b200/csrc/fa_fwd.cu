@@ -169,24 +169,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
   if (warp == C::kLoadWarp) {
     // Union list of this range's key tiles needed by either query tile, with per-tile keep
     // bits; entries hold the K/V tile index, the masks see its query-sequence tile jg.
-    int count = 0, c0 = 0, c1 = 0;
+    int c0, c1;
     const int jb = split * a.split_tiles;
-    const int je = min(a.Tk, jb + a.split_tiles);
-    for (int base = jb; base < je; base += 32) {
-      const int j = base + lane;
-      bool k0 = false, k1 = false;
-      if (j < je) {
-        const int qa = qt0, qb = qt0 + 1, jg = a.kt_off + j;
-        k0 = (!a.causal || jg <= qa) && (a.blockmask == nullptr || a.blockmask[(size_t)qa * a.T + jg] != 0);
-        k1 = kQ == 2 && qb < a.T && (!a.causal || jg <= qb) &&
-             (a.blockmask == nullptr || a.blockmask[(size_t)qb * a.T + jg] != 0);
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, k0 || k1);
-      if (k0 || k1) list[count + __popc(bal & ((1u << lane) - 1u))] = j | (int(k0) << 16) | (int(k1) << 17);
-      count += __popc(bal);
-      c0 += __popc(__ballot_sync(0xffffffffu, k0));
-      c1 += __popc(__ballot_sync(0xffffffffu, k1));
-    }
+    const int count = union_tile_list(list, jb, min(a.Tk, jb + a.split_tiles), a.kt_off, qt0, kQ == 2, a.T, a.causal,
+                                      a.blockmask, c0, c1);
     if (lane == 0) {
       sh.n_union = count;
       sh.n_q[0] = c0;
@@ -425,16 +411,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kQ>::kThreads, kQ == 2 ? 1 : 2)
         for (int i = 0; i < 128; ++i)
           if (i >= lim) s[i] = -INFINITY;
       }
-      // Row max: eight independent chains of 3-input maxima (depth 10 instead of a 127-long
-      // dependent chain), then one combine.
-      float mxa[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mxa[k] = fmaxf(s[2 * k], s[2 * k + 1]);
-#pragma unroll
-      for (int i = 16; i < 128; i += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mxa[k] = max3f(mxa[k], s[i + 2 * k], s[i + 2 * k + 1]);
-      const float mx = max3f(max3f(mxa[0], mxa[1], mxa[2]), max3f(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
+      const float mx = row_max128(s);
       const float mx2 = mx * sl2;
       float alpha = 1.f;
       bool resc = false;

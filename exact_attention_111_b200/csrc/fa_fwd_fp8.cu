@@ -162,22 +162,8 @@ __global__ void __launch_bounds__(320, 1)
   }
   if (warp == 8) {
     // Union list of key tiles needed by either query tile, with per-tile keep bits.
-    int count = 0, c0 = 0, c1 = 0;
-    for (int base = 0; base < a.T; base += 32) {
-      const int j = base + lane;
-      bool k0 = false, k1 = false;
-      if (j < a.T) {
-        const int qa = qt0, qb = qt0 + 1;
-        k0 = (!a.causal || j <= qa) && (a.blockmask == nullptr || a.blockmask[(size_t)qa * a.T + j] != 0);
-        k1 = qb < a.T && (!a.causal || j <= qb) &&
-             (a.blockmask == nullptr || a.blockmask[(size_t)qb * a.T + j] != 0);
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, k0 || k1);
-      if (k0 || k1) list[count + __popc(bal & ((1u << lane) - 1u))] = j | (int(k0) << 16) | (int(k1) << 17);
-      count += __popc(bal);
-      c0 += __popc(__ballot_sync(0xffffffffu, k0));
-      c1 += __popc(__ballot_sync(0xffffffffu, k1));
-    }
+    int c0, c1;
+    const int count = union_tile_list(list, 0, a.T, 0, qt0, true, a.T, a.causal, a.blockmask, c0, c1);
     if (lane == 0) {
       sh.n_union = count;
       sh.n_q[0] = c0;
@@ -327,14 +313,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < 128; ++i)
           if (i >= lim) s[i] = -INFINITY;
       }
-      float mxa[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mxa[k] = fmaxf(s[2 * k], s[2 * k + 1]);
-#pragma unroll
-      for (int i = 16; i < 128; i += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mxa[k] = max3f(mxa[k], s[i + 2 * k], s[i + 2 * k + 1]);
-      const float mx = max3f(max3f(mxa[0], mxa[1], mxa[2]), max3f(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
+      const float mx = row_max128(s);
       const float mx2 = mx * sl2;
       float alpha = 1.f;
       bool resc = false;

@@ -351,6 +351,47 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return m;
 }
 
+// Max of one 128-score row: eight independent chains of 3-input maxima (depth 10 instead of a
+// 127-long dependent chain), then one combine.
+__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+  float mxa[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mxa[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+  for (int i = 16; i < 128; i += 16)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mxa[k] = max3f(mxa[k], s[i + 2 * k], s[i + 2 * k + 1]);
+  return max3f(max3f(mxa[0], mxa[1], mxa[2]), max3f(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
+}
+
+// The forward's list of key tiles for a CTA: tiles j in [jb, je) that query tile qt0, or qt0
+// and qt0 + 1 (two), keep; entry = j | keep0 << 16 | keep1 << 17.  Tile j sits at query-sequence
+// tile kt_off + j: causal keeps it iff that is <= the query tile, a block mask [T][T] iff its
+// entry is nonzero.  One warp builds the list (a ballot per 32 tiles); every lane gets the number
+// of entries (returned) and of tiles each query tile keeps (n0, n1).
+__device__ __forceinline__ int union_tile_list(int* list, int jb, int je, int kt_off, int qt0, bool two, int T,
+                                               bool causal, const uint8_t* mask, int& n0, int& n1) {
+  const int lane = threadIdx.x & 31;
+  int count = 0;
+  n0 = 0;
+  n1 = 0;
+  for (int base = jb; base < je; base += 32) {
+    const int j = base + lane;
+    bool k0 = false, k1 = false;
+    if (j < je) {
+      const int qa = qt0, qb = qt0 + 1, jg = kt_off + j;
+      k0 = (!causal || jg <= qa) && (mask == nullptr || mask[(size_t)qa * T + jg] != 0);
+      k1 = two && qb < T && (!causal || jg <= qb) && (mask == nullptr || mask[(size_t)qb * T + jg] != 0);
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, k0 || k1);
+    if (k0 || k1) list[count + __popc(bal & ((1u << lane) - 1u))] = j | (int(k0) << 16) | (int(k1) << 17);
+    count += __popc(bal);
+    n0 += __popc(__ballot_sync(0xffffffffu, k0));
+    n1 += __popc(__ballot_sync(0xffffffffu, k1));
+  }
+  return count;
+}
+
 // Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction for two lanes of math).
 __device__ __forceinline__ unsigned long long f2pack(float a, float b) {
   unsigned long long r;
